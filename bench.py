@@ -1,0 +1,349 @@
+"""Benchmark of the ISA forward pass on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one ISA forward call over the headline workload (B=1, H=40, D=128,
+L_src = L_ctx = 16384, b = 128, alpha_s = 0.25, alpha_f = 0.6: the 32K-token
+case), inputs resident in HBM. `value` is the effective throughput in TFLOP/s
+(FLOPs the pass executes: coarse scores, routing, exact and Taylor attention)
+over all ranks; `ms_per_step` is the max over ranks. Under torchrun each rank
+runs its own replica of the workload (independent batches: weak scaling, no
+collective on the data path; NCCL only for the barrier and the max of the
+timings).
+
+`--impl reference` times the CPU oracle (float64 numpy) as it stands on the
+host cores over a bounded sample of the same workload (one head per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import isa_synth  # noqa: E402
+
+METRIC = "ISA forward ms/call and effective TFLOPS at 32K tokens; fraction of roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+# ----------------------------------------------------------------------------- host-side logic (tested on CPU)
+
+def flops_per_call(w) -> dict:
+    """Multiply-adds of each stage x 2 for one call over all B*H slices (the pass's own counts)."""
+    N = w.L_src + w.L_ctx
+    n_q, n_src, n_ctx = N // w.b, w.L_src // w.b, w.L_ctx // w.b
+    k = max(0, min(n_ctx, math.ceil(float(np.float32(w.alpha_s)) * n_ctx - 1e-4)))
+    n_flat = max(0, min(n_q, math.floor(float(np.float32(w.alpha_f)) * n_q + 1e-4)))
+    n_new = n_src + k
+    bh = w.B * w.H
+    f = dict(coarse=2.0 * n_src * n_q * w.D * bh, route=2.0 * n_q * n_new * w.D * bh,
+             exact=4.0 * (n_q - n_flat) * w.b * n_new * w.b * w.D * bh,
+             taylor=4.0 * n_flat * w.b * n_new * w.D * bh)
+    f["total"] = sum(f.values())
+    return f
+
+
+def hbm_bytes_per_call(w) -> dict:
+    """Algorithmic HBM bytes of the pooling/top-k stage (read Q, K, V once) and the gather."""
+    e = 2 if w.dtype == "bf16" else 4
+    N = w.L_src + w.L_ctx
+    n_ctx = w.L_ctx // w.b
+    k = max(0, min(n_ctx, math.ceil(float(np.float32(w.alpha_s)) * n_ctx - 1e-4)))
+    return dict(pool=3.0 * w.B * w.H * N * w.D * e, gather=2.0 * 2.0 * w.B * w.H * k * w.b * w.D * e)
+
+
+def reduce_max(x: float, dist=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    if dist is None or not dist.is_initialized():
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(flops_per_rank: float, max_ms: float, world: int) -> float:
+    """Whole-job TFLOP/s: all ranks' FLOPs over the slowest rank's time."""
+    return flops_per_rank * world / (max_ms * 1e-3) / 1e12
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except FileNotFoundError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.flush()
+        with open(self.f.name) as g:
+            rows = [r.strip().split(", ") for r in g if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, pw, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                pw.append(float(r[3]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        busy = [s for s, p in zip(sm, pw) if p > 200] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None, "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- arms
+
+def workload_inputs(w, seed=0):
+    att = isa_synth.attempts_for(w, seed)
+    return isa_synth.make_inputs(w, seed, att)
+
+
+def bf16_bits(x):
+    return isa_synth.round_to_bf16_bits(x)
+
+
+def cpu_oracle_sample(w, q, k, v, heads, seconds_cap=60.0):
+    """Run the oracle on some heads; returns (TFLOP/s, seconds, heads done)."""
+    from oracle import isa_oracle as O
+    f = flops_per_call(w)["total"] / (w.B * w.H)
+    t0 = time.perf_counter()
+    done = 0
+    for h in heads:
+        O.isa_slice_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+        done += 1
+        if time.perf_counter() - t0 > seconds_cap:
+            break
+    dt = time.perf_counter() - t0
+    return f * done / dt / 1e12, dt, done
+
+
+def run_reference(args, w):
+    """The CPU oracle as it stands, one head of the workload per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    q, k, v = isa_synth.make_inputs(w, 0, isa_synth.attempts_for(w, 0), heads=[(0, h) for h in range(w.H)][:max(1, args.steps + args.warmup)])
+    from oracle import isa_oracle as O
+    f_head = flops_per_call(w)["total"] / (w.B * w.H)
+    for s in range(args.warmup):
+        O.isa_slice_ref(q[0, s % w.H], k[0, s % w.H], v[0, s % w.H], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        h = (args.warmup + s) % w.H
+        O.isa_slice_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+    dt = time.perf_counter() - t0
+    value = f_head * args.steps / dt / 1e12
+    cores = os.cpu_count()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "b": w.b,
+                       "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "sample": "one head per step"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} heads of {w.B * w.H}, one per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_isa_b200 as isa
+    from block_sparse_attention_isa_b200 import build as isa_build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=300))
+    isa_build.build()
+    dev = torch.device("cuda", local)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    q, k, v = workload_inputs(w)
+    tq, tk, tv = (torch.from_numpy(x).to(dev, dt) for x in (q, k, v))
+    out = torch.empty_like(tq)
+    ws = torch.empty(isa.workspace_bytes(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s,
+                                         isa.ISA_BF16 if w.dtype == "bf16" else isa.ISA_F32),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        isa.forward_into(tq, tk, tv, out, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    isa.device_status(ws, stream)
+
+    # per-kernel events for every timed step
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(args.steps):
+        isa.set_stage_events(ev[s])
+        step()
+    end.record(stream)
+    isa.set_stage_events(None)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    isa.device_status(ws, stream)
+
+    ms = start.elapsed_time(end) / args.steps
+    max_ms = reduce_max(ms, dist)
+    stage_ms = {name: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)) / args.steps
+                for i, name in enumerate(isa.STAGES)}
+    f = flops_per_call(w)
+    hb = hbm_bytes_per_call(w)
+    peaks, peaks_kind = load_peaks()
+    attn_tflops = (f["exact"] + f["taylor"]) / (stage_ms["attention"] * 1e-3) / 1e12
+    peak_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    pool_gbs = hb["pool"] / (stage_ms["pool_score_topk"] * 1e-3) / 1e9
+    gather_gbs = hb["gather"] / max(stage_ms["gather"] * 1e-3, 1e-12) / 1e9
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        with open(prof) as fh:
+            traffic = json.load(fh).get(w.name, {}).get("attention")
+
+    # end to end through the host-buffer entry point (pinned host memory, copies inside the timed region)
+    e2e = None
+    if rank == 0 or world > 1:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (tq, tk, tv))
+        hout = torch.empty_like(hq).pin_memory()
+        n_e2e = max(1, min(args.steps, 5))
+        isa.forward_host(hq, hk, hv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, out=hout)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(n_e2e):
+            isa.forward_host(hq, hk, hv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, out=hout)
+        e2e_ms = (time.perf_counter() - t0) / n_e2e * 1e3
+        e2e_ms = reduce_max(e2e_ms, dist)
+        nbytes = hq.numel() * hq.element_size()
+        e2e = {"value": aggregate(f["total"], e2e_ms, world), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, secs, done = cpu_oracle_sample(w, q, k, v, heads=range(w.H), seconds_cap=args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+               "sample": f"{done} of {w.B * w.H} heads of the same workload, {secs:.1f} s of CPU time"}
+
+    launches = isa.launch_count(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, w.alpha_f,
+                                isa.ISA_BF16 if w.dtype == "bf16" else isa.ISA_F32)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": aggregate(f["total"], max_ms, world), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "b": w.b,
+                       "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "global_batch": w.B * world,
+                       "seq_len": w.N, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (Q, K, V = %.2f GB per step)" % (3 * tq.numel() * tq.element_size() / 1e9)},
+            "roofline": {"bound": "tensor", "kernel": "attention (exact + Taylor paths)", "achieved": attn_tflops,
+                         "peak": peak_sust, "unit": "TFLOP/s", "frac": attn_tflops / peak_sust,
+                         "peak_kind": f"{peaks_kind} bf16 sustained",
+                         "frac_of_burst": attn_tflops / peaks["bf16_tflops"], "traffic": traffic},
+            "stages_ms": stage_ms,
+            "hbm_stages": {"pool_score_topk_gbs": pool_gbs, "gather_gbs": gather_gbs,
+                           "pool_frac": pool_gbs / peaks["hbm_gbs"], "gather_frac": gather_gbs / peaks["hbm_gbs"],
+                           "peak_gbs": peaks["hbm_gbs"], "peak_kind": peaks_kind},
+            "flops_per_call": f,
+            "gpu_launches": launches * args.steps,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=isa_synth.HEADLINE)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = isa_synth.all_workloads()[args.workload]
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

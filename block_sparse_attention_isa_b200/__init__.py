@@ -1,0 +1,299 @@
+"""In-context Sparse Attention (ISA) forward pass for NVIDIA B200 (sm_100a).
+
+Python binding of the C-ABI library ``libisa.so`` (declared in
+``include/isa.h``). The binding only marshals arguments: every step of the
+pass runs in the library's CUDA kernels. PyTorch provides device memory and
+streams. There is no CPU fallback; if the library is missing this module
+raises on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+__all__ = [
+    "IsaError",
+    "ISA_BF16",
+    "ISA_F32",
+    "lib",
+    "lib_path",
+    "plan",
+    "workspace_bytes",
+    "launch_count",
+    "forward",
+    "forward_into",
+    "forward_host",
+    "device_status",
+    "debug_pooled",
+    "selftest_wait_timeout",
+    "set_stage_events",
+    "STAGES",
+    "last_error",
+    "EXPORTS",
+]
+
+ISA_BF16 = 0
+ISA_F32 = 1
+
+ERROR_NAMES = {
+    0: "ISA_OK",
+    -1: "ISA_ERR_ARG",
+    -2: "ISA_ERR_SHAPE",
+    -3: "ISA_ERR_UNSUPPORTED",
+    -4: "ISA_ERR_WORKSPACE",
+    -5: "ISA_ERR_CUDA",
+    -6: "ISA_ERR_TIMEOUT",
+}
+
+# Every function declared in include/isa.h.
+EXPORTS = (
+    "isa_plan",
+    "isa_workspace_bytes",
+    "isa_forward_ex",
+    "isa_forward",
+    "isa_forward_host",
+    "isa_device_status",
+    "isa_debug_pooled",
+    "isa_launch_count",
+    "isa_selftest_wait_timeout",
+    "isa_set_stage_events",
+    "isa_last_error",
+)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+class IsaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{ERROR_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libisa.so")
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libisa.so (built in-tree by ``python -m block_sparse_attention_isa_b200.build``)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = os.environ.get("ISA_LIBRARY_PATH") or lib_path()
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m block_sparse_attention_isa_b200.build`")
+    L = ctypes.CDLL(path)
+    c_int, c_float, c_size, vp = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    fp = ctypes.POINTER(ctypes.c_float)
+    L.isa_plan.argtypes = [c_int] * 6 + [c_float, c_float, i32p, i32p, i32p]
+    L.isa_plan.restype = c_int
+    L.isa_workspace_bytes.argtypes = [c_int] * 6 + [c_float, c_int]
+    L.isa_workspace_bytes.restype = c_size
+    L.isa_forward_ex.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_float, c_int, vp, vp, vp, vp, c_size, vp]
+    L.isa_forward_ex.restype = c_int
+    L.isa_forward.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_float, vp, vp, vp]
+    L.isa_forward.restype = c_int
+    L.isa_forward_host.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_float, c_int, vp, vp, vp]
+    L.isa_forward_host.restype = c_int
+    L.isa_device_status.argtypes = [vp, vp]
+    L.isa_device_status.restype = c_int
+    L.isa_debug_pooled.argtypes = [c_int] * 6 + [c_float, c_int, vp, vp, vp, vp, vp, vp, vp]
+    L.isa_debug_pooled.restype = c_int
+    L.isa_launch_count.argtypes = [c_int] * 6 + [c_float, c_float, c_int]
+    L.isa_launch_count.restype = c_int
+    L.isa_selftest_wait_timeout.argtypes = [vp, c_int, vp]
+    L.isa_selftest_wait_timeout.restype = c_int
+    L.isa_set_stage_events.argtypes = [vp, c_int]
+    L.isa_set_stage_events.restype = c_int
+    L.isa_last_error.argtypes = []
+    L.isa_last_error.restype = ctypes.c_char_p
+    _LIB = L
+    return L
+
+
+def last_error() -> str:
+    return lib().isa_last_error().decode()
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise IsaError(rc, last_error())
+
+
+def plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f) -> Tuple[int, int, int]:
+    """(n_q, k, n_flat) for these sizes: query blocks, kept context blocks, Taylor blocks."""
+    n_q, k, n_flat = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().isa_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, ctypes.byref(n_q), ctypes.byref(k),
+                          ctypes.byref(n_flat)))
+    return n_q.value, k.value, n_flat.value
+
+
+def workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dtype=ISA_BF16) -> int:
+    n = lib().isa_workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dtype)
+    if n == 0:
+        raise IsaError(-1, last_error())
+    return n
+
+
+def launch_count(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dtype=ISA_BF16) -> int:
+    return lib().isa_launch_count(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dtype)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return ISA_BF16
+    if t.dtype == torch.float32:
+        return ISA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+_WS_CACHE = {}
+
+
+def _workspace(device, nbytes: int):
+    torch = _torch()
+    key = (device.index if device.index is not None else torch.cuda.current_device())
+    ws = _WS_CACHE.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _WS_CACHE[key] = ws
+    return ws
+
+
+def forward_into(q, k, v, out, L_src: int, L_ctx: int, b: int, alpha_s: float, alpha_f: float,
+                 dbg_sel=None, dbg_route=None, workspace=None, stream=None):
+    """Enqueue the pass on ``stream`` (default: torch's current stream) writing ``out``.
+
+    All tensors are CUDA tensors; q, k, v, out are contiguous [B, H, N, D] of one
+    dtype (bfloat16 or float32); dbg_sel int32 [B, H, k] and dbg_route int32
+    [B, H, n_q] are optional. Asynchronous; returns the workspace used.
+    """
+    torch = _torch()
+    for t in (q, k, v, out):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("q, k, v and out must be contiguous 4-D CUDA tensors [B, H, N, D]")
+    B, H, N, D = q.shape
+    dt = _dtype_code(q)
+    if workspace is None:
+        workspace = _workspace(q.device, workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dt))
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    s = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    rc = lib().isa_forward_ex(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dt, out.data_ptr(),
+        dbg_sel.data_ptr() if dbg_sel is not None else None, dbg_route.data_ptr() if dbg_route is not None else None,
+        workspace.data_ptr(), workspace.numel(), s)
+    _check(rc)
+    return workspace
+
+
+def forward(q, k, v, L_src: int, L_ctx: int, b: int, alpha_s: float, alpha_f: float, debug: bool = False,
+            stream=None):
+    """ISA forward pass on CUDA tensors; returns out, or (out, sel, route) when ``debug``."""
+    torch = _torch()
+    out = torch.empty_like(q)
+    sel = route = None
+    if debug:
+        B, H, N, D = q.shape
+        n_q, kk, _ = plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f)
+        sel = torch.empty((B, H, kk), dtype=torch.int32, device=q.device)
+        route = torch.empty((B, H, n_q), dtype=torch.int32, device=q.device)
+    forward_into(q, k, v, out, L_src, L_ctx, b, alpha_s, alpha_f, sel, route, stream=stream)
+    return (out, sel, route) if debug else out
+
+
+def device_status(workspace=None, stream=None):
+    """Synchronise and raise IsaError(ISA_ERR_TIMEOUT) if a kernel wait gave up."""
+    torch = _torch()
+    if workspace is None:
+        dev = torch.cuda.current_device()
+        workspace = _WS_CACHE.get(dev)
+        if workspace is None:
+            return
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device)
+    s = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    _check(lib().isa_device_status(workspace.data_ptr(), s))
+
+
+STAGES = ("pool_score_topk", "gather", "route", "attention")
+
+
+def set_stage_events(events):
+    """Record these 5 torch.cuda.Event objects around the 4 kernels of the next calls (None to stop)."""
+    if events is None:
+        _check(lib().isa_set_stage_events(None, 0))
+        return
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _check(lib().isa_set_stage_events(arr, len(events)))
+
+
+def selftest_wait_timeout(workspace, timeout_ms: int = 100, stream=None):
+    """Enqueue a kernel whose wait can never complete; its bounded wait gives up and flags ``workspace``."""
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device)
+    s = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    _check(lib().isa_selftest_wait_timeout(workspace.data_ptr(), timeout_ms, s))
+
+
+def debug_pooled(B, H, L_src, L_ctx, D, b, alpha_s, dtype=ISA_BF16, workspace=None, stream=None):
+    """Intermediates of the last call made with ``workspace``: dict of Qc, Kc, Vc, colscore, sharp."""
+    torch = _torch()
+    n_q = (L_src + L_ctx) // b
+    dev = torch.cuda.current_device() if workspace is None else workspace.device
+    if workspace is None:
+        workspace = _WS_CACHE[dev]
+    f = dict(device=workspace.device, dtype=torch.float32)
+    res = dict(qc=torch.empty((B, H, n_q, D), **f), kc=torch.empty((B, H, n_q, D), **f),
+               vc=torch.empty((B, H, n_q, D), **f), colscore=torch.empty((B, H, L_ctx // b), **f),
+               sharp=torch.empty((B, H, n_q), **f))
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device)
+    s = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    _check(lib().isa_debug_pooled(B, H, L_src, L_ctx, D, b, alpha_s, dtype, workspace.data_ptr(),
+                                  res["qc"].data_ptr(), res["kc"].data_ptr(), res["vc"].data_ptr(),
+                                  res["colscore"].data_ptr(), res["sharp"].data_ptr(), s))
+    return res
+
+
+def forward_host(q, k, v, L_src: int, L_ctx: int, b: int, alpha_s: float, alpha_f: float, out=None,
+                 dbg_sel=None, dbg_route=None, dtype: Optional[int] = None):
+    """The pass on HOST buffers (numpy arrays or CPU tensors, pinned or not): copies in, runs, copies out.
+
+    For bfloat16, pass uint16 numpy arrays holding the bit patterns, or bfloat16 CPU tensors.
+    """
+    import numpy as np
+
+    def ptr(a):
+        if a is None:
+            return None
+        if isinstance(a, np.ndarray):
+            if not a.flags["C_CONTIGUOUS"]:
+                raise ValueError("host arrays must be C-contiguous")
+            return a.ctypes.data
+        if not a.is_contiguous() or a.is_cuda:
+            raise ValueError("host tensors must be contiguous CPU tensors")
+        return a.data_ptr()
+
+    B, H, N, D = q.shape
+    if dtype is None:
+        if isinstance(q, np.ndarray):
+            dtype = ISA_F32 if q.dtype == np.float32 else ISA_BF16
+        else:
+            dtype = _dtype_code(q)
+    if out is None:
+        out = np.empty_like(q) if isinstance(q, np.ndarray) else _torch().empty_like(q)
+    _check(lib().isa_forward_host(ptr(q), ptr(k), ptr(v), B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dtype,
+                                  ptr(out), ptr(dbg_sel), ptr(dbg_route)))
+    return out

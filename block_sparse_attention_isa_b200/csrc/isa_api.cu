@@ -1,0 +1,376 @@
+// C ABI of the In-context Sparse Attention forward pass: argument checks,
+// block counts, workspace layout and the stream-ordered launch sequence
+//   pool + coarse score + top-k  ->  gather  ->  sharpness + routing  ->  attention.
+// See include/isa.h for the contract of every entry point.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/isa.h"
+#include "isa_internal.h"
+
+namespace isa {
+
+namespace {
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(ISA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Kept context blocks: ceil(alpha_s * n_ctx) with a 1e-4 guard on the float ratio.
+int kept_blocks(float alpha_s, int n_ctx) {
+  const double x = (double)alpha_s * (double)n_ctx;
+  long kk = (long)std::ceil(x - 1e-4);
+  if (kk < 0) kk = 0;
+  if (kk > n_ctx) kk = n_ctx;
+  return (int)kk;
+}
+// Taylor query blocks: floor(alpha_f * n_q) with a 1e-4 guard on the float ratio.
+int flat_blocks(float alpha_f, int n_q) {
+  const double x = (double)alpha_f * (double)n_q;
+  long n = (long)std::floor(x + 1e-4);
+  if (n < 0) n = 0;
+  if (n > n_q) n = n_q;
+  return (int)n;
+}
+
+bool ratio_ok(float a) { return !std::isnan(a) && a >= 0.0f && a <= 1.0f; }
+
+int make_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, int dt, Plan* p) {
+  if (B <= 0 || H <= 0) return fail(ISA_ERR_ARG, "B and H must be positive (B=%d H=%d)", B, H);
+  if (L_src <= 0 || L_ctx <= 0) return fail(ISA_ERR_ARG, "L_src and L_ctx must be positive (%d, %d)", L_src, L_ctx);
+  if (!ratio_ok(alpha_s) || !ratio_ok(alpha_f))
+    return fail(ISA_ERR_ARG, "alpha_s and alpha_f must lie in [0, 1] (%g, %g)", (double)alpha_s, (double)alpha_f);
+  if (dt != ISA_BF16 && dt != ISA_F32) return fail(ISA_ERR_UNSUPPORTED, "unknown dtype %d", dt);
+  if (D != 64 && D != 128) return fail(ISA_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
+  if (b != 64 && b != 128) return fail(ISA_ERR_UNSUPPORTED, "block size b must be 64 or 128 (got %d)", b);
+  if (dt == ISA_F32 && D != 64) return fail(ISA_ERR_UNSUPPORTED, "float32 inputs need D = 64");
+  if (L_src % b || L_ctx % b)
+    return fail(ISA_ERR_SHAPE, "L_src (%d) and L_ctx (%d) must be multiples of b (%d)", L_src, L_ctx, b);
+  const long long N = (long long)L_src + L_ctx;
+  if (N > (1ll << 30)) return fail(ISA_ERR_UNSUPPORTED, "N too large");
+  const long long BH = (long long)B * H;
+  if (BH > 65535) return fail(ISA_ERR_UNSUPPORTED, "B*H must be at most 65535");
+  const int n_q = (int)(N / b);
+  if (n_q > kMaxBlocks) return fail(ISA_ERR_UNSUPPORTED, "N / b must be at most %d (got %d)", kMaxBlocks, n_q);
+  p->B = B;
+  p->H = H;
+  p->BH = (int)BH;
+  p->N = (int)N;
+  p->D = D;
+  p->b = b;
+  p->L_src = L_src;
+  p->L_ctx = L_ctx;
+  p->n_q = n_q;
+  p->n_src = L_src / b;
+  p->n_ctx = L_ctx / b;
+  p->k = kept_blocks(alpha_s, p->n_ctx);
+  p->n_new = p->n_src + p->k;
+  p->L_new = p->n_new * b;
+  p->n_flat = flat_blocks(alpha_f, n_q);
+  p->n_exact = n_q - p->n_flat;
+  p->dt = dt;
+  p->elem = dt == ISA_BF16 ? 2 : 4;
+  return ISA_OK;
+}
+
+bool overlaps(const void* a, const void* b, size_t bytes) {
+  const char* x = static_cast<const char*>(a);
+  const char* y = static_cast<const char*>(b);
+  return x < y + bytes && y < x + bytes;
+}
+
+}  // namespace
+
+size_t workspace_layout(const Plan& p, Work* w, char* base) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* r = base ? base + off : nullptr;
+    off += align256(bytes);
+    return r;
+  };
+  const size_t BH = p.BH;
+  Work t{};
+  t.ctrl = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * (kCtrlWords + 2 * BH)));
+  if (base) {
+    t.ctr_pool = t.ctrl + kCtrlWords;
+    t.ctr_route = t.ctr_pool + BH;
+  }
+  t.qc = reinterpret_cast<float*>(take(sizeof(float) * BH * p.n_q * p.D));
+  t.kc = reinterpret_cast<float*>(take(sizeof(float) * BH * p.n_q * p.D));
+  t.vc = reinterpret_cast<float*>(take(sizeof(float) * BH * p.n_q * p.D));
+  t.colscore = reinterpret_cast<float*>(take(sizeof(float) * BH * p.n_ctx));
+  t.sel = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * BH * (p.k > 0 ? p.k : 1)));
+  t.sharp = reinterpret_cast<float*>(take(sizeof(float) * BH * p.n_q));
+  t.route = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * BH * p.n_q));
+  t.kcn = take((size_t)p.elem * BH * p.n_new * p.D);
+  t.vcn = take((size_t)p.elem * BH * p.n_new * p.D);
+  t.ksel = take((size_t)p.elem * BH * (p.k > 0 ? p.k : 1) * p.b * p.D);
+  t.vsel = take((size_t)p.elem * BH * (p.k > 0 ? p.k : 1) * p.b * p.D);
+  if (w) *w = t;
+  return off;
+}
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+// Optional CUDA events recorded between the stages of the next forward calls on
+// this host thread (set by isa_set_stage_events; used for live per-kernel timing).
+thread_local cudaEvent_t g_stage_events[kStageEvents] = {};
+thread_local bool g_stage_events_on = false;
+
+inline cudaError_t mark(int i, cudaStream_t s) {
+  return g_stage_events_on ? cudaEventRecord(g_stage_events[i], s) : cudaSuccess;
+}
+
+int run_forward(const void* q, const void* k, const void* v, const Plan& p, void* out, int32_t* dbg_sel,
+                int32_t* dbg_route, void* workspace, size_t workspace_bytes, cudaStream_t s) {
+  const size_t need = workspace_layout(p, nullptr, nullptr);
+  if (!workspace) return fail(ISA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+  if (workspace_bytes < need)
+    return fail(ISA_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(ISA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  Work w;
+  workspace_layout(p, &w, static_cast<char*>(workspace));
+  cudaError_t e = cudaMemsetAsync(w.ctrl, 0, sizeof(uint32_t) * (kCtrlWords + 2 * (size_t)p.BH), s);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace counters");
+  if ((e = mark(0, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
+  if ((e = launch_pool_score_topk(q, k, v, p, w, s)) != cudaSuccess) return cuda_fail(e, "pool/score/top-k launch");
+  if ((e = mark(1, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
+  if ((e = launch_gather(k, v, p, w, s)) != cudaSuccess) return cuda_fail(e, "gather launch");
+  if ((e = mark(2, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
+  if ((e = launch_route(p, w, s)) != cudaSuccess) return cuda_fail(e, "routing launch");
+  if ((e = mark(3, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
+  if ((e = launch_attention(q, k, v, out, p, w, s, nullptr)) != cudaSuccess) return cuda_fail(e, "attention launch");
+  if ((e = mark(4, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
+  if (dbg_sel && p.k > 0) {
+    e = cudaMemcpyAsync(dbg_sel, w.sel, sizeof(int32_t) * (size_t)p.BH * p.k, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copying dbg_sel");
+  }
+  if (dbg_route) {
+    e = cudaMemcpyAsync(dbg_route, w.route, sizeof(int32_t) * (size_t)p.BH * p.n_q, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copying dbg_route");
+  }
+  return ISA_OK;
+}
+
+int check_io(const void* q, const void* k, const void* v, const void* out, const Plan& p) {
+  if (!q || !k || !v || !out) return fail(ISA_ERR_ARG, "q, k, v and out must not be NULL");
+  const size_t bytes = (size_t)p.BH * p.N * p.D * p.elem;
+  if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes))
+    return fail(ISA_ERR_ARG, "out must not overlap q, k or v");
+  return ISA_OK;
+}
+
+int read_status(void* workspace, cudaStream_t s) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "synchronising the stream");
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (word) {
+    cudaMemset(workspace, 0, sizeof(word));
+    return fail(ISA_ERR_TIMEOUT, "a kernel wait timed out (error word 0x%x)", word);
+  }
+  return ISA_OK;
+}
+
+}  // namespace
+}  // namespace isa
+
+using namespace isa;
+
+extern "C" {
+
+const char* isa_last_error(void) { return g_err; }
+
+int isa_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, int32_t* n_q,
+             int32_t* k, int32_t* n_flat) {
+  Plan p;
+  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, ISA_BF16, &p);
+  if (rc != ISA_OK) return rc;
+  if (n_q) *n_q = p.n_q;
+  if (k) *k = p.k;
+  if (n_flat) *n_flat = p.n_flat;
+  return ISA_OK;
+}
+
+size_t isa_workspace_bytes(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, isa_dtype dt) {
+  Plan p;
+  if (make_plan(B, H, L_src, L_ctx, D, b, alpha_s, 0.0f, (int)dt, &p) != ISA_OK) return 0;
+  return workspace_layout(p, nullptr, nullptr);
+}
+
+int isa_launch_count(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, isa_dtype dt) {
+  Plan p;
+  if (make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p) != ISA_OK) return 0;
+  return 3 + (p.k > 0 ? 1 : 0);
+}
+
+int isa_forward_ex(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
+                   float alpha_s, float alpha_f, isa_dtype dt, void* out, int32_t* dbg_sel, int32_t* dbg_route,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  Plan p;
+  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p);
+  if (rc != ISA_OK) return rc;
+  if ((rc = check_io(q, k, v, out, p)) != ISA_OK) return rc;
+  return run_forward(q, k, v, p, out, dbg_sel, dbg_route, workspace, workspace_bytes,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int isa_forward(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
+                float alpha_s, float alpha_f, void* out, int32_t* dbg_sel, int32_t* dbg_route) {
+  Plan p;
+  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, ISA_BF16, &p);
+  if (rc != ISA_OK) return rc;
+  if ((rc = check_io(q, k, v, out, p)) != ISA_OK) return rc;
+  const size_t ws_bytes = workspace_layout(p, nullptr, nullptr);
+  void* ws = nullptr;
+  cudaStream_t s = 0;
+  cudaError_t e = cudaMallocAsync(&ws, ws_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "allocating the workspace");
+  rc = run_forward(q, k, v, p, out, dbg_sel, dbg_route, ws, ws_bytes, s);
+  const int st = read_status(ws, s);
+  if (rc == ISA_OK) rc = st;
+  cudaFreeAsync(ws, s);
+  e = cudaStreamSynchronize(s);
+  if (rc == ISA_OK && e != cudaSuccess) rc = cuda_fail(e, "freeing the workspace");
+  return rc;
+}
+
+int isa_forward_host(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
+                     float alpha_s, float alpha_f, isa_dtype dt, void* out, int32_t* dbg_sel, int32_t* dbg_route) {
+  Plan p;
+  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p);
+  if (rc != ISA_OK) return rc;
+  if ((rc = check_io(q, k, v, out, p)) != ISA_OK) return rc;
+  const size_t io = align256((size_t)p.BH * p.N * p.D * p.elem);
+  const size_t ws_bytes = workspace_layout(p, nullptr, nullptr);
+  const size_t sel_b = align256(sizeof(int32_t) * (size_t)p.BH * (p.k > 0 ? p.k : 1));
+  const size_t route_b = align256(sizeof(int32_t) * (size_t)p.BH * p.n_q);
+  const size_t total = 4 * io + ws_bytes + sel_b + route_b;
+  cudaStream_t s = 0;
+  // keep freed blocks in the stream-ordered pool so that repeated calls do not
+  // go back to the driver for memory
+  int dev = 0;
+  cudaMemPool_t pool;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+    uint64_t thr = UINT64_MAX;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
+  }
+  char* dev_buf = nullptr;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&dev_buf), total, s);
+  if (e != cudaSuccess) return cuda_fail(e, "allocating device buffers");
+  char* dq = dev_buf;
+  char* dk = dq + io;
+  char* dv = dk + io;
+  char* dout = dv + io;
+  char* dws = dout + io;
+  int32_t* dsel = reinterpret_cast<int32_t*>(dws + ws_bytes);
+  int32_t* droute = reinterpret_cast<int32_t*>(dws + ws_bytes + sel_b);
+  const size_t bytes = (size_t)p.BH * p.N * p.D * p.elem;
+  rc = ISA_OK;
+  if ((e = cudaMemcpyAsync(dq, q, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dk, k, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dv, v, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+    rc = cuda_fail(e, "copying inputs to the device");
+  if (rc == ISA_OK)
+    rc = run_forward(dq, dk, dv, p, dout, dbg_sel ? dsel : nullptr, dbg_route ? droute : nullptr, dws, ws_bytes, s);
+  if (rc == ISA_OK && (e = cudaMemcpyAsync(out, dout, bytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    rc = cuda_fail(e, "copying the output to the host");
+  if (rc == ISA_OK && dbg_sel && p.k > 0 &&
+      (e = cudaMemcpyAsync(dbg_sel, dsel, sizeof(int32_t) * (size_t)p.BH * p.k, cudaMemcpyDeviceToHost, s)) !=
+          cudaSuccess)
+    rc = cuda_fail(e, "copying dbg_sel to the host");
+  if (rc == ISA_OK && dbg_route &&
+      (e = cudaMemcpyAsync(dbg_route, droute, sizeof(int32_t) * (size_t)p.BH * p.n_q, cudaMemcpyDeviceToHost, s)) !=
+          cudaSuccess)
+    rc = cuda_fail(e, "copying dbg_route to the host");
+  const int st = read_status(dws, s);
+  if (rc == ISA_OK) rc = st;
+  cudaFreeAsync(dev_buf, s);
+  e = cudaStreamSynchronize(s);
+  if (rc == ISA_OK && e != cudaSuccess) rc = cuda_fail(e, "releasing device buffers");
+  return rc;
+}
+
+int isa_selftest_wait_timeout(void* workspace, int timeout_ms, void* stream) {
+  if (!workspace) return fail(ISA_ERR_WORKSPACE, "workspace is NULL");
+  if (timeout_ms <= 0 || timeout_ms > 10000) return fail(ISA_ERR_ARG, "timeout_ms must lie in [1, 10000]");
+  cudaError_t e = launch_wait_selftest(static_cast<uint32_t*>(workspace), timeout_ms, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return ISA_OK;
+}
+
+int isa_set_stage_events(void* const* events, int n_events) {
+  if (!events) {
+    g_stage_events_on = false;
+    return ISA_OK;
+  }
+  if (n_events != kStageEvents) return fail(ISA_ERR_ARG, "exactly %d events are needed", kStageEvents);
+  for (int i = 0; i < kStageEvents; ++i) {
+    if (!events[i]) return fail(ISA_ERR_ARG, "event %d is NULL", i);
+    g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  g_stage_events_on = true;
+  return ISA_OK;
+}
+
+int isa_device_status(void* workspace, void* stream) {
+  if (!workspace) return fail(ISA_ERR_WORKSPACE, "workspace is NULL");
+  return read_status(workspace, static_cast<cudaStream_t>(stream));
+}
+
+int isa_debug_pooled(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, isa_dtype dt,
+                     const void* workspace, float* qc, float* kc, float* vc, float* colscore, float* sharp,
+                     void* stream) {
+  Plan p;
+  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, 0.0f, (int)dt, &p);
+  if (rc != ISA_OK) return rc;
+  if (!workspace) return fail(ISA_ERR_WORKSPACE, "workspace is NULL");
+  Work w;
+  workspace_layout(p, &w, static_cast<char*>(const_cast<void*>(workspace)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t pooled = sizeof(float) * (size_t)p.BH * p.n_q * p.D;
+  struct {
+    float* dst;
+    const float* src;
+    size_t bytes;
+  } cp[5] = {{qc, w.qc, pooled},
+             {kc, w.kc, pooled},
+             {vc, w.vc, pooled},
+             {colscore, w.colscore, sizeof(float) * (size_t)p.BH * p.n_ctx},
+             {sharp, w.sharp, sizeof(float) * (size_t)p.BH * p.n_q}};
+  for (auto& c : cp) {
+    if (!c.dst) continue;
+    cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copying pooled intermediates");
+  }
+  return ISA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// Internal types shared by the ISA kernels and the C-ABI layer.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace isa {
+
+// Sizes of one call, all derived on the host from the arguments.
+struct Plan {
+  int B, H, BH, N, D, b, L_src, L_ctx;
+  int n_q;     // N / b query blocks (also key blocks)
+  int n_src;   // L_src / b
+  int n_ctx;   // L_ctx / b
+  int k;       // kept context blocks
+  int n_new;   // n_src + k blocks in K_new
+  int L_new;   // n_new * b keys in K_new
+  int n_flat;  // query blocks on the Taylor path
+  int n_exact; // n_q - n_flat query blocks on the exact path
+  int dt;      // 0 = bf16, 1 = fp32
+  int elem;    // bytes per element
+};
+
+// Views into the caller's workspace (all 256-byte aligned).
+struct Work {
+  uint32_t* ctrl;        // [kCtrlWords]: error word, spare words
+  uint32_t* ctr_pool;    // [BH] CTAs of the pooling grid finished per head
+  uint32_t* ctr_route;   // [BH] CTAs of the routing grid finished per head
+  float* qc;             // [BH, n_q, D] block means of Q (fp32)
+  float* kc;             // [BH, n_q, D]
+  float* vc;             // [BH, n_q, D]
+  float* colscore;       // [BH, n_ctx] context-block scores
+  int32_t* sel;          // [BH, max(k,1)] kept context blocks, ascending
+  float* sharp;          // [BH, n_q] query-block sharpness M_i
+  int32_t* route;        // [BH, n_q] exact blocks ascending, then Taylor blocks ascending
+  void* kcn;             // [BH, n_new, D] pooled K_new blocks in the MMA element type
+  void* vcn;             // [BH, n_new, D]
+  void* ksel;            // [BH, k*b, D] gathered context keys
+  void* vsel;            // [BH, k*b, D]
+};
+
+constexpr int kCtrlWords = 64;
+constexpr int kStageEvents = 5;  // before pooling, after pooling, gather, routing, attention
+constexpr int kMaxBlocks = 2048;  // max n_q supported by the per-head sorts
+
+// Error-word bits written by kernels when a bounded wait gives up.
+enum : uint32_t {
+  kErrProducer = 1u << 0,
+  kErrMma = 1u << 1,
+  kErrSoftmax = 1u << 2,
+  kErrGather = 1u << 3,
+  kErrSelftest = 1u << 4,
+};
+
+size_t workspace_layout(const Plan& p, Work* w, char* base);
+
+cudaError_t launch_pool_score_topk(const void* q, const void* k, const void* v, const Plan& p, const Work& w,
+                                   cudaStream_t s);
+cudaError_t launch_gather(const void* k, const void* v, const Plan& p, const Work& w, cudaStream_t s);
+cudaError_t launch_route(const Plan& p, const Work& w, cudaStream_t s);
+cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out, const Plan& p,
+                             const Work& w, cudaStream_t s, int* n_ctas_out);
+
+// One thread waits on an mbarrier that nothing arrives on; the bounded wait gives
+// up after `timeout_ms` and sets kErrSelftest in err[0].
+cudaError_t launch_wait_selftest(uint32_t* err, int timeout_ms, cudaStream_t s);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace isa

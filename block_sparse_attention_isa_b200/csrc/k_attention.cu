@@ -1,0 +1,602 @@
+// Stage 4-5 of In-context Sparse Attention: both attention paths and the
+// write-back, as one persistent tcgen05 kernel.
+//
+// Method: "Lightning Unified Video Editing via In-Context Sparse Attention",
+// papernotes.org notes, Key design 2 and the flowchart:
+//  * exact path (sharp query blocks): S = Q K_new^T / sqrt(D), P = exp(S),
+//    l += rowsum(P), O += P V_new, O /= l, by online softmax over all keys of
+//    K_new = [K_src ; kept context blocks];
+//  * block-wise 0th-order Taylor path (flat query blocks): each block j of
+//    K_new stands in as b * exp(q . Kc_j / sqrt(D)) paired with Vc_j. Every
+//    block holds b keys, so the weight b cancels between numerator and
+//    denominator and the path is softmax(q Kc_new^T / sqrt(D)) Vc_new: the same
+//    online-softmax attention, against the n_new pooled rows instead of L_new
+//    keys. The paperlayer.ai summary, section 3 (Taylor Sparse Attention),
+//    gives the O(L_Q D) cost per query block that this reaches;
+//  * each output row is written at its original token position (each query
+//    block takes exactly one path, so there is nothing to merge).
+//
+// Design for sm_100a (prior art on the pages is Triton / TileLang on Hopper):
+//  * one CTA per SM (persistent), 12 warps: warp 0 issues TMA loads, warp 1
+//    owns TMEM and issues tcgen05.mma from one thread (warps 2-3 idle), warps
+//    4-7 and 8-11 are two softmax warpgroups, one per 128-row query tile;
+//    each softmax thread owns one query row and keeps its 128 scores in
+//    registers (setmaxnreg moves registers from warpgroup 0 to them);
+//  * a work item is up to two 128-row query tiles of one head (four blocks
+//    when b = 64), both walking the same K/V tiles, so every K/V tile is
+//    loaded once for 256 query rows;
+//  * TMEM: S_t at columns [128 t, 128 t + 128), O_t at [256 + 128 t, ...);
+//    P_t is written over S_t (bf16 pairs, or fp32 for tf32) and fed to the
+//    P V MMA straight from TMEM;
+//  * MMA order per K/V tile j: PV0_j, S0_{j+1}, PV1_j, S1_{j+1}, so the tensor
+//    core works on one tile while the softmax warps work on the other;
+//  * lazy rescaling: the running max only moves when it grows by more than
+//    2^8, and only then is the O row rescaled in TMEM by its own thread;
+//  * exact items come first in the static schedule and Taylor items after.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <float.h>
+
+#include "isa_internal.h"
+#include "ptx.cuh"
+
+namespace isa {
+namespace {
+
+constexpr int kThreads = 384;  // 3 warpgroups
+// Register budget: the kernel is compiled for 168 registers a thread at launch
+// (384 x 168 = 64512 of the SM's 65536). Warpgroup 0 (TMA + MMA warps) gives
+// registers back and the two softmax warpgroups take them:
+// 128 x 56 + 256 x 224 = 64512, the same total, so the increase never waits.
+// The launcher checks the compiled count before every launch.
+constexpr int kLaunchRegs = 168;
+constexpr int kLowRegs = 56;
+constexpr int kHighRegs = 224;
+static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per K/V tile
+constexpr float kRescaleThreshold = 8.0f;  // log2 domain
+
+struct AttnParams {
+  const int32_t* route;
+  void* out;
+  uint32_t* err;
+  int BH, N, b, L_src, n_q, n_exact, n_flat, L_new, n_new;
+  int bpt;       // blocks per 128-row tile (128 / b)
+  int bpi;       // blocks per item (2 tiles)
+  int items_e;   // exact items per head
+  int items_t;   // Taylor items per head
+  int total;     // all items
+  float scale_log2;
+};
+
+template <typename T, int D>
+struct Cfg {
+  static constexpr int E = sizeof(T);
+  static constexpr bool kTf32 = (E == 4);
+  static constexpr int RB = D * E;              // bytes per row
+  static constexpr int NCH = RB / 128;          // 128-byte swizzle chunks per row
+  static constexpr int CH_STRIDE = kBM * 128;   // bytes between chunks of a 128-row tile
+  static constexpr int TILE = kBM * RB;         // bytes of one 128-row tile
+  static constexpr int BOX_X = 128 / E;         // elements per 128-byte chunk row
+  static constexpr int KS_QK = RB / 32;         // UMMA K-steps of Q K^T (32 bytes each)
+  static constexpr int PV_K = 32 / E;           // keys per P V UMMA
+  static constexpr int KS_PV = kBN / PV_K;
+  static constexpr int STAGES = 2;
+  static constexpr uint32_t FMT = kTf32 ? 2u : 1u;
+  static constexpr uint32_t IDESC_QK = umma_idesc(FMT, kBM, kBN, 0, 0);
+  static constexpr uint32_t IDESC_PV = umma_idesc(FMT, kBM, D, 0, 1);
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = 2 * TILE;
+  static constexpr int OFF_V = OFF_K + STAGES * TILE;
+  static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
+  static constexpr int SMEM_USED = OFF_BAR + 256;
+  // padded above half of the SM's shared memory so that exactly one CTA (and one
+  // 512-column TMEM allocation) lives on each SM
+  static constexpr int SMEM_ALLOC = (SMEM_USED + 1024 > 120 * 1024 ? SMEM_USED + 1024 : 120 * 1024);
+  static_assert(NCH >= 1 && NCH <= 2, "row of 128 or 256 bytes");
+  static_assert(D % 32 == 0, "D multiple of 32");
+};
+
+struct Item {
+  int bh, kind, nblk, ntiles, nkv, last_valid;
+  int blk0, blk1, blk2, blk3;  // query blocks of the item (repeats of blk0 past nblk)
+  __device__ __forceinline__ int blk(int u) const { return u == 0 ? blk0 : u == 1 ? blk1 : u == 2 ? blk2 : blk3; }
+};
+
+__device__ __forceinline__ Item decode_item(const AttnParams& p, int g) {
+  Item it;
+  int count, base, pp;
+  if (g < p.BH * p.items_e) {
+    it.bh = g / p.items_e;
+    pp = g - it.bh * p.items_e;
+    it.kind = 0;
+    count = p.n_exact;
+    base = 0;
+  } else {
+    const int g2 = g - p.BH * p.items_e;
+    it.bh = g2 / p.items_t;
+    pp = g2 - it.bh * p.items_t;
+    it.kind = 1;
+    count = p.n_flat;
+    base = p.n_exact;
+  }
+  const int32_t* lst = p.route + (size_t)it.bh * p.n_q + base;
+  const int first = pp * p.bpi;
+  it.nblk = min(p.bpi, count - first);
+  it.blk0 = __ldg(lst + first);
+  it.blk1 = it.nblk > 1 ? __ldg(lst + first + 1) : it.blk0;
+  it.blk2 = it.nblk > 2 ? __ldg(lst + first + 2) : it.blk0;
+  it.blk3 = it.nblk > 3 ? __ldg(lst + first + 3) : it.blk0;
+  it.ntiles = (it.nblk + p.bpt - 1) / p.bpt;
+  const int rows = it.kind == 0 ? p.L_new : p.n_new;
+  it.nkv = (rows + kBN - 1) / kBN;
+  it.last_valid = rows - kBN * (it.nkv - 1);
+  return it;
+}
+
+struct Bars {
+  uint64_t q_full[2];
+  uint64_t q_empty;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], p_ready[2], o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ bool aborted(const Bars* b) {
+  return *reinterpret_cast<const volatile int*>(&b->abort_flag) != 0;
+}
+__device__ __forceinline__ void raise_abort(Bars* b, uint32_t* err, uint32_t code) {
+  atomicOr(err, code);
+  *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
+}
+
+// All 32 lanes wait on the barrier; the result is the same in every lane and the
+// warp is converged on return (the TMEM moves that follow are warp-collective).
+__device__ __forceinline__ bool warp_wait(Bars* b, uint64_t* bar, uint32_t parity, uint32_t* err) {
+  bool ok = !aborted(b) && mbar_wait(bar, parity);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok) raise_abort(b, err, kErrSoftmax);
+  tc_fence_after();
+  return ok;
+}
+
+template <typename T>
+__device__ __forceinline__ void store_row_chunk(T* dst, const float* v);  // 32 values
+
+template <>
+__device__ __forceinline__ void store_row_chunk<__nv_bfloat16>(__nv_bfloat16* dst, const float* v) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    pk[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+}
+template <>
+__device__ __forceinline__ void store_row_chunk<float>(float* dst, const float* v) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_ksel, const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_vsel, const __grid_constant__ CUtensorMap tm_kcn,
+                     const __grid_constant__ CUtensorMap tm_vcn, const AttnParams p) {
+  using C = Cfg<T, D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->q_full[t], 1);
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_ready[t], 128);
+      mbar_init(&bars->o_done[t], 1);
+    }
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_ksel);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_vsel);
+    tma_prefetch_desc(&tm_kcn);
+    tma_prefetch_desc(&tm_vcn);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 4) regs_dealloc<kLowRegs>();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t kv_it = 0, n_local = 0;
+      uint32_t q_arm[2] = {0, 0};
+      uint32_t k_arm[C::STAGES] = {}, v_arm[C::STAGES] = {};
+      bool ok = true;
+      for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x, ++n_local) {
+        const Item it = decode_item(p, g);
+        if (n_local > 0 && !mbar_wait(&bars->q_empty, (n_local - 1) & 1)) {
+          raise_abort(bars, p.err, kErrProducer);
+          ok = false;
+          break;
+        }
+        for (int t = 0; t < it.ntiles; ++t) {
+          mbar_arrive_expect_tx(&bars->q_full[t], C::TILE);
+          ++q_arm[t];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int r = 64 * h;
+            int u = t * p.bpt + r / p.b;
+            if (u >= it.nblk) u = t * p.bpt;  // missing block: load a valid one, rows are not stored
+            const int y = it.blk(u) * p.b + (r % p.b);
+#pragma unroll
+            for (int c = 0; c < C::NCH; ++c)
+              tma_load_3d(sQ + t * C::TILE + c * C::CH_STRIDE + h * 8192, &tm_q, &bars->q_full[t], c * C::BOX_X,
+                          y, it.bh);
+          }
+        }
+        for (int j = 0; j < it.nkv; ++j, ++kv_it) {
+          if (aborted(bars)) { ok = false; break; }
+          const int st = kv_it % C::STAGES;
+          const uint32_t ph = (kv_it / C::STAGES) & 1;
+          // K tile
+          if (!mbar_wait(&bars->k_empty[st], ph ^ 1)) { raise_abort(bars, p.err, kErrProducer); ok = false; break; }
+          mbar_arrive_expect_tx(&bars->k_full[st], C::TILE);
+          ++k_arm[st];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int r0 = j * kBN + 64 * h;
+            const CUtensorMap* map;
+            int y;
+            if (it.kind == 0) {
+              if (r0 < p.L_src) { map = &tm_k; y = r0; } else { map = &tm_ksel; y = r0 - p.L_src; }
+            } else {
+              map = &tm_kcn; y = r0;
+            }
+#pragma unroll
+            for (int c = 0; c < C::NCH; ++c)
+              tma_load_3d(sK + st * C::TILE + c * C::CH_STRIDE + h * 8192, map, &bars->k_full[st], c * C::BOX_X,
+                          y, it.bh);
+          }
+          // V tile
+          if (!mbar_wait(&bars->v_empty[st], ph ^ 1)) { raise_abort(bars, p.err, kErrProducer); ok = false; break; }
+          mbar_arrive_expect_tx(&bars->v_full[st], C::TILE);
+          ++v_arm[st];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int r0 = j * kBN + 64 * h;
+            const CUtensorMap* map;
+            int y;
+            if (it.kind == 0) {
+              if (r0 < p.L_src) { map = &tm_v; y = r0; } else { map = &tm_vsel; y = r0 - p.L_src; }
+            } else {
+              map = &tm_vcn; y = r0;
+            }
+#pragma unroll
+            for (int c = 0; c < C::NCH; ++c)
+              tma_load_3d(sV + st * C::TILE + c * C::CH_STRIDE + h * 8192, map, &bars->v_full[st], c * C::BOX_X,
+                          y, it.bh);
+          }
+        }
+      }
+      if (!ok) {
+        // let every copy this thread started land before the CTA can leave
+        for (int t = 0; t < 2; ++t)
+          if (q_arm[t]) mbar_wait(&bars->q_full[t], (q_arm[t] - 1) & 1);
+        for (int s = 0; s < C::STAGES; ++s) {
+          if (k_arm[s]) mbar_wait(&bars->k_full[s], (k_arm[s] - 1) & 1);
+          if (v_arm[s]) mbar_wait(&bars->v_full[s], (v_arm[s] - 1) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t kv_it = 0;
+      uint32_t q_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
+      bool ok = true;
+      const uint32_t sq = smem_addr(sQ), sk = smem_addr(sK), sv = smem_addr(sV);
+      auto issue_s = [&](int t, int st) {
+        const uint32_t d = tmem + t * 128;
+        const uint32_t qa = sq + t * C::TILE, ka = sk + st * C::TILE;
+#pragma unroll
+        for (int s = 0; s < C::KS_QK; ++s) {
+          const uint32_t off = (s / 4) * C::CH_STRIDE + (s % 4) * 32;
+          umma_ss<C::kTf32>(d, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), C::IDESC_QK,
+                            s > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int st, bool acc) {
+        const uint32_t d = tmem + 256 + t * 128;
+        const uint32_t pa = tmem + t * 128;
+        const uint32_t va = sv + st * C::TILE;
+#pragma unroll
+        for (int s = 0; s < C::KS_PV; ++s)
+          umma_ts<C::kTf32>(d, pa + s * 8, smem_desc_sw128(va + s * C::PV_K * 128, C::CH_STRIDE, 1024), C::IDESC_PV,
+                            (acc || s > 0) ? 1u : 0u);
+      };
+      auto wait_or_abort = [&](uint64_t* bar, uint32_t par) -> bool {
+        if (aborted(bars)) { ok = false; return false; }
+        if (!mbar_wait(bar, par)) { raise_abort(bars, p.err, kErrMma); ok = false; return false; }
+        tc_fence_after();
+        return true;
+      };
+      for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x) {
+        const Item it = decode_item(p, g);
+        for (int t = 0; t < it.ntiles; ++t) {
+          if (!wait_or_abort(&bars->q_full[t], q_cnt[t] & 1)) break;
+          ++q_cnt[t];
+        }
+        if (!ok) break;
+        // S_t for the first K/V tile
+        {
+          const int st = kv_it % C::STAGES;
+          if (!wait_or_abort(&bars->k_full[st], (kv_it / C::STAGES) & 1)) break;
+          for (int t = 0; t < it.ntiles; ++t) {
+            issue_s(t, st);
+            umma_commit(&bars->s_full[t]);
+          }
+          umma_commit(&bars->k_empty[st]);
+          if (it.nkv == 1) umma_commit(&bars->q_empty);
+        }
+        for (int j = 0; j < it.nkv && ok; ++j, ++kv_it) {
+          const int st = kv_it % C::STAGES;
+          if (!wait_or_abort(&bars->v_full[st], (kv_it / C::STAGES) & 1)) break;
+          const bool more = (j + 1 < it.nkv);
+          const int st1 = (kv_it + 1) % C::STAGES;
+          for (int t = 0; t < it.ntiles; ++t) {
+            if (!wait_or_abort(&bars->p_ready[t], pv_cnt[t] & 1)) break;
+            issue_pv(t, st, j > 0);
+            umma_commit(&bars->o_done[t]);
+            ++pv_cnt[t];
+            if (more) {
+              if (t == 0 && !wait_or_abort(&bars->k_full[st1], ((kv_it + 1) / C::STAGES) & 1)) break;
+              issue_s(t, st1);
+              umma_commit(&bars->s_full[t]);
+              if (t == it.ntiles - 1) {
+                umma_commit(&bars->k_empty[st1]);
+                if (j + 2 == it.nkv) umma_commit(&bars->q_empty);
+              }
+            }
+          }
+          if (!ok) break;
+          umma_commit(&bars->v_empty[st]);
+        }
+      }
+      // every MMA issued by this thread completes before TMEM can be released
+      umma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    regs_alloc<kHighRegs>();
+    const int t = (warp - 4) >> 2;           // query tile of this warpgroup
+    const int wl = warp & 3;                 // TMEM lane quarter
+    const int row = wl * 32 + lane;          // row inside the 128-row tile
+    const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + t * 128;
+    const uint32_t t_o = tmem + lane_off + 256 + t * 128;
+    uint32_t s_cnt = 0, pv_cnt = 0;
+    bool ok = true;
+    T* out = static_cast<T*>(p.out);
+    for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x) {
+      const Item it = decode_item(p, g);
+      if (t >= it.ntiles) continue;
+      float m = -FLT_MAX, l = 0.f;
+      for (int j = 0; j < it.nkv; ++j) {
+        if (!warp_wait(bars, &bars->s_full[t], s_cnt & 1, p.err)) { ok = false; break; }
+        ++s_cnt;
+        uint32_t r[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, r + 32 * c);
+        tmem_ld_wait<128>(r);
+        const int valid = (j == it.nkv - 1) ? it.last_valid : kBN;
+        float mx = -FLT_MAX;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          float x = __uint_as_float(r[i]) * p.scale_log2;
+          x = (i < valid) ? x : -FLT_MAX;
+          r[i] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+        // lazy max: move it only when the tile's max exceeds it by more than 2^8
+        const bool need = (j > 0) && (mx > m + kRescaleThreshold);
+        const float alpha = need ? ex2_approx(m - mx) : 1.0f;
+        if (j == 0 || need) m = mx;
+        float rs = 0.f;
+        if constexpr (sizeof(T) == 2) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const float p0 = ex2_approx(__uint_as_float(r[2 * i]) - m);
+            const float p1 = ex2_approx(__uint_as_float(r[2 * i + 1]) - m);
+            rs += p0 + p1;
+            __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+            r[i] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          tmem_st32(t_s, r);
+          tmem_st32(t_s + 32, r + 32);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) {
+            const float pv = ex2_approx(__uint_as_float(r[i]) - m);
+            rs += pv;
+            r[i] = __float_as_uint(pv);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_st32(t_s + 32 * c, r + 32 * c);
+        }
+        l = l * alpha + rs;
+        // O holds P V up to tile j-1; rows whose max moved are rescaled in place
+        // before P V of tile j may start. TMEM moves are warp-collective, so the
+        // whole warp takes this step when any of its rows needs it (alpha = 1 for
+        // the others).
+        if (__any_sync(0xffffffffu, need)) {
+          if (!warp_wait(bars, &bars->o_done[t], (pv_cnt - 1) & 1, p.err)) { ok = false; break; }
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + 32 * c, o);
+            tmem_ld_wait<32>(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_o + 32 * c, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->p_ready[t]);
+        ++pv_cnt;
+      }
+      if (!ok) break;
+      // epilogue: O / l written at the row's original token position
+      if (!warp_wait(bars, &bars->o_done[t], (pv_cnt - 1) & 1, p.err)) { ok = false; break; }
+      const float inv_l = 1.0f / l;
+      const int u = t * p.bpt + row / p.b;
+      const bool store = (u < it.nblk);
+      const size_t token = (size_t)it.blk(store ? u : 0) * p.b + (row % p.b);
+      T* dst = out + ((size_t)it.bh * p.N + token) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + 32 * c, o);
+        tmem_ld_wait<32>(o);
+        float* f = reinterpret_cast<float*>(o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(o[i]) * inv_l;
+        if (store) store_row_chunk<T>(dst + 32 * c, f);
+      }
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [heads][rows][D] view, box of 64 rows x one 128-byte chunk, 128-byte swizzle,
+// out-of-range rows read as zeros.
+bool make_map(CUtensorMap* m, const void* base, int elem, int D, int rows, int heads) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const CUtensorMapDataType dt = elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)D * elem, (cuuint64_t)rows * D * elem};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / elem), 64u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const void* q, const void* k, const void* v, void* out, const Plan& pl, const Work& w,
+                     cudaStream_t s, int* n_ctas) {
+  using C = Cfg<T, D>;
+  AttnParams p{};
+  p.route = w.route;
+  p.out = out;
+  p.err = w.ctrl;
+  p.BH = pl.BH;
+  p.N = pl.N;
+  p.b = pl.b;
+  p.L_src = pl.L_src;
+  p.n_q = pl.n_q;
+  p.n_exact = pl.n_exact;
+  p.n_flat = pl.n_flat;
+  p.L_new = pl.L_new;
+  p.n_new = pl.n_new;
+  p.bpt = kBM / pl.b;
+  p.bpi = 2 * p.bpt;
+  p.items_e = (pl.n_exact + p.bpi - 1) / p.bpi;
+  p.items_t = (pl.n_flat + p.bpi - 1) / p.bpi;
+  p.total = pl.BH * (p.items_e + p.items_t);
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  if (n_ctas) *n_ctas = 0;
+  if (p.total == 0) return cudaSuccess;
+
+  const int E = sizeof(T);
+  CUtensorMap tq, tk, tks, tv, tvs, tkc, tvc;
+  const bool has_sel = pl.k > 0;
+  if (!make_map(&tq, q, E, D, pl.N, pl.BH) || !make_map(&tk, k, E, D, pl.N, pl.BH) ||
+      !make_map(&tv, v, E, D, pl.N, pl.BH) ||
+      !make_map(&tks, has_sel ? w.ksel : k, E, D, has_sel ? pl.k * pl.b : pl.N, pl.BH) ||
+      !make_map(&tvs, has_sel ? w.vsel : v, E, D, has_sel ? pl.k * pl.b : pl.N, pl.BH) ||
+      !make_map(&tkc, w.kcn, E, D, pl.n_new, pl.BH) || !make_map(&tvc, w.vcn, E, D, pl.n_new, pl.BH))
+    return cudaErrorInvalidValue;
+
+  auto kern = attention_kernel<T, D>;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  // the warpgroup register split is only safe with the launch count it was sized for
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  int grid = device_sm_count();
+  if (grid > p.total) grid = p.total;
+  kern<<<grid, kThreads, C::SMEM_ALLOC, s>>>(tq, tk, tks, tv, tvs, tkc, tvc, p);
+  if (n_ctas) *n_ctas = grid;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out, const Plan& p, const Work& w,
+                             cudaStream_t s, int* n_ctas) {
+  if (p.dt == 0) return p.D == 128 ? launch_t<__nv_bfloat16, 128>(q, k, v, out, p, w, s, n_ctas)
+                                   : launch_t<__nv_bfloat16, 64>(q, k, v, out, p, w, s, n_ctas);
+  if (p.D == 64) return launch_t<float, 64>(q, k, v, out, p, w, s, n_ctas);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace isa

@@ -1,0 +1,175 @@
+/*
+ * isa.h - C ABI of the In-context Sparse Attention (ISA) forward pass for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method is the one of "Lightning Unified Video Editing via In-Context
+ * Sparse Attention" (arXiv 2605.04569), as described in the papernotes.org
+ * notes (Overall framework; Key designs 1-3) and the paperlayer.ai summary
+ * (sections 2 and 3). For an in-context sequence whose first L_src tokens are
+ * the source video and whose last L_ctx tokens are the context, one call runs:
+ *
+ *   1. pooling probe: Qc, Kc, Vc = means over blocks of b tokens;
+ *      S_coarse = softmax(Qc Kc^T / sqrt(D)) over all n_q = N / b key blocks
+ *      (papernotes, Key design 1; paperlayer, section 2 "Pooling Attention");
+ *   2. context pre-selection: score[c] = mean over the source query blocks of
+ *      S_coarse[i, n_src + c]; keep the k = ceil(alpha_s * L_ctx / b) best
+ *      context blocks and gather K_new = [K_src ; kept blocks], same for V
+ *      (papernotes, Key design 1; paperlayer, section 3 "Pre-Selection");
+ *   3. sharpness routing: M_i = Var(softmax(Qc_i Kc_new^T / sqrt(D))); the
+ *      floor(alpha_f * n_q) blocks of lowest M_i take the approximate path
+ *      (papernotes, Key design 3; paperlayer, section 3 "Grouped Computation");
+ *   4. exact attention over K_new / V_new for the other blocks, and block-wise
+ *      0th-order Taylor attention (each K_new block stands in as its mean key
+ *      with weight b and its mean value) for the flat blocks (papernotes, Key
+ *      design 2);
+ *   5. both outputs written back in the original token order.
+ *
+ * Readings where the pages are silent (they are fixed here, and the CPU
+ * oracle of the test suite follows the same ones): L_src and L_ctx are
+ * multiples of b; k = ceil(alpha_s * n_ctx - 1e-4) and
+ * n_flat = floor(alpha_f * n_q + 1e-4), computed in double from the float
+ * arguments; top-k and routing ties break by lower block index; kept blocks
+ * enter K_new in ascending order after the source part.
+ *
+ * Layout: q, k, v and out are row-major contiguous [B, H, N, D] with
+ * N = L_src + L_ctx, in the element type given by isa_dtype (bfloat16 or
+ * float32); out has the same type. Sizes supported: D in {64, 128}, b in
+ * {64, 128}, N / b <= 2048; float32 only with D = 64.
+ *
+ * Ownership: the caller owns every buffer passed in. The library never frees
+ * caller memory and keeps no pointer after a call returns.
+ *
+ * Errors: a negative return code, never an exception or an abort. The
+ * thread-local message of the last failure is available from
+ * isa_last_error().
+ */
+#ifndef ISA_H
+#define ISA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ISA_API __attribute__((visibility("default")))
+#else
+#define ISA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { ISA_BF16 = 0, ISA_F32 = 1 } isa_dtype;
+
+enum {
+  ISA_OK = 0,
+  ISA_ERR_ARG = -1,         /* null or aliased pointer, non-positive size, ratio outside [0,1] or NaN */
+  ISA_ERR_SHAPE = -2,       /* L_src or L_ctx not a multiple of b */
+  ISA_ERR_UNSUPPORTED = -3, /* D, b, dtype or N / b outside the supported set */
+  ISA_ERR_WORKSPACE = -4,   /* workspace null or smaller than isa_workspace_bytes() */
+  ISA_ERR_CUDA = -5,        /* a CUDA runtime error; the message holds cudaGetErrorString() */
+  ISA_ERR_TIMEOUT = -6      /* a kernel's bounded wait gave up (reported by isa_device_status) */
+};
+
+/*
+ * isa_plan - block counts of a call, computed on the host only (no CUDA).
+ * Writes n_q (query / key blocks), k (kept context blocks) and n_flat (Taylor
+ * query blocks); any output pointer may be NULL. Returns ISA_OK or an error
+ * code for invalid arguments (same checks as isa_forward_ex).
+ */
+ISA_API int isa_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f,
+             int32_t* n_q, int32_t* k, int32_t* n_flat);
+
+/*
+ * isa_workspace_bytes - device workspace size that isa_forward_ex needs for
+ * these sizes (0 if the arguments are invalid; the reason is in
+ * isa_last_error()). The workspace holds the pooled blocks, the coarse
+ * scores, the selection and routing lists and the gathered context blocks.
+ */
+ISA_API size_t isa_workspace_bytes(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, isa_dtype dt);
+
+/*
+ * isa_forward_ex - the whole forward pass, enqueued on `stream`
+ * (a cudaStream_t; NULL = the legacy default stream). Asynchronous: returns
+ * once the kernels are enqueued. All pointers are device pointers.
+ *   q, k, v      [B, H, N, D] inputs (read only, must not alias out)
+ *   out          [B, H, N, D] output
+ *   dbg_sel      optional int32 [B, H, k]: kept context blocks (0-based,
+ *                relative to the first context block), ascending; NULL to skip
+ *   dbg_route    optional int32 [B, H, n_q]: exact-path blocks ascending,
+ *                then Taylor-path blocks ascending; NULL to skip
+ *   workspace    device memory of at least isa_workspace_bytes(), 256-byte
+ *                aligned, used as scratch; it must not be shared by calls that
+ *                may run at the same time
+ * The enqueue makes no device->host synchronisation and no allocation.
+ */
+ISA_API int isa_forward_ex(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
+                   float alpha_s, float alpha_f, isa_dtype dt, void* out, int32_t* dbg_sel, int32_t* dbg_route,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * isa_forward - bfloat16 convenience form: allocates its workspace with
+ * cudaMallocAsync on the legacy default stream, runs isa_forward_ex, checks
+ * the device status, frees the workspace and synchronises before returning.
+ */
+ISA_API int isa_forward(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
+                float alpha_s, float alpha_f, void* out, int32_t* dbg_sel, int32_t* dbg_route);
+
+/*
+ * isa_forward_host - the same pass with HOST buffers (pageable or pinned):
+ * copies q, k, v to the device, runs the pass, copies out (and the optional
+ * dbg_sel / dbg_route, host int32) back, then synchronises. Device memory is
+ * allocated and freed inside the call. Element type as given by dt.
+ */
+ISA_API int isa_forward_host(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
+                     float alpha_s, float alpha_f, isa_dtype dt, void* out, int32_t* dbg_sel, int32_t* dbg_route);
+
+/*
+ * isa_device_status - synchronises `stream`, then reads and clears the error
+ * word that kernels of earlier calls with this workspace may have set.
+ * Returns ISA_OK, ISA_ERR_TIMEOUT (a bounded wait in a kernel gave up) or
+ * ISA_ERR_CUDA.
+ */
+ISA_API int isa_device_status(void* workspace, void* stream);
+
+/*
+ * isa_debug_pooled - copies intermediates of the LAST isa_forward_ex call made
+ * with this workspace (stream-ordered on `stream`): qc, kc, vc as float32
+ * [B, H, n_q, D], colscore float32 [B, H, n_ctx], sharp float32 [B, H, n_q].
+ * Any output pointer may be NULL. The sizes must match that call.
+ */
+ISA_API int isa_debug_pooled(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, isa_dtype dt,
+                     const void* workspace, float* qc, float* kc, float* vc, float* colscore, float* sharp,
+                     void* stream);
+
+/*
+ * isa_selftest_wait_timeout - enqueues a one-thread kernel that waits on a
+ * barrier nothing will ever arrive on. Its bounded wait gives up after
+ * timeout_ms (1..10000) and sets the error word of `workspace` (at least 256
+ * bytes of device memory, e.g. a forward workspace), so that the next
+ * isa_device_status on it returns ISA_ERR_TIMEOUT. It exercises the same
+ * bounded-wait path that guards every wait of the forward kernels, without
+ * faulting or hanging the GPU, and leaves the CUDA context usable.
+ */
+ISA_API int isa_selftest_wait_timeout(void* workspace, int timeout_ms, void* stream);
+
+/*
+ * isa_set_stage_events - for live per-kernel timing: while set, every forward
+ * call made on this host thread records the 5 given CUDA events (cudaEvent_t
+ * handles owned by the caller) on its stream: before the pooling kernel and
+ * after the pooling, gather, routing and attention kernels. Pass NULL to stop.
+ * Returns ISA_ERR_ARG unless n_events == 5 and no handle is NULL.
+ */
+ISA_API int isa_set_stage_events(void* const* events, int n_events);
+
+/* Number of kernel launches one isa_forward_ex call makes for these sizes (0 if invalid). */
+ISA_API int isa_launch_count(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, isa_dtype dt);
+
+/* Message of the last failed call on this host thread ("" if none). */
+ISA_API const char* isa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISA_H */

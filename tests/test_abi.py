@@ -1,0 +1,112 @@
+"""Host-side tests of the C ABI: build, symbol exports, argument checks, block counts.
+
+No test here launches a kernel: every call either fails its host-side checks
+before touching CUDA, or only computes sizes. Fake device addresses are only
+ever passed together with a missing or undersized workspace, which the library
+rejects before any CUDA call.
+"""
+import ctypes
+import math
+import os
+import re
+import subprocess
+
+import pytest
+
+import isa_synth
+import block_sparse_attention_isa_b200 as isa
+from oracle import isa_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "isa.h")
+FAKE = 0x7F0000000000  # never dereferenced: every call below fails its checks first
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_sparse_attention_isa_b200 import build
+    build.build()
+    return isa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(isa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(isa.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", isa.lib_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (isa_[a-z_]+)\b", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(L, name) is not None
+    # nothing else leaks from the library's C++ internals
+    assert all(n.startswith("isa_") for n in exported)
+
+
+@pytest.mark.parametrize("name", sorted(isa_synth.all_workloads()))
+def test_block_counts_match_oracle(L, name):
+    w = isa_synth.all_workloads()[name]
+    n_q, k, n_flat = isa.plan(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, w.alpha_f)
+    assert n_q == w.N // w.b
+    assert k == O.kept_context_blocks(w.alpha_s, w.L_ctx // w.b)
+    assert n_flat == O.taylor_block_count(w.alpha_f, n_q)
+
+
+def test_headline_counts():
+    assert isa.plan(1, 40, 16384, 16384, 128, 128, 0.25, 0.6) == (256, 32, 153)
+    # float32 0.1 * 200 = 20.0000003 must not round up to 21
+    assert isa.plan(1, 40, 25600, 25600, 128, 128, 0.1, 0.3) == (400, 20, 120)
+
+
+def _fwd(L, q=FAKE, k=FAKE, v=FAKE, B=1, H=2, L_src=512, L_ctx=512, D=64, b=64, a_s=0.5, a_f=0.5, dt=0,
+         out=FAKE + (1 << 32), ws=None, ws_bytes=0):
+    return L.isa_forward_ex(q, k, v, B, H, L_src, L_ctx, D, b, a_s, a_f, dt, out, None, None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(k=None), -1), (dict(v=None), -1), (dict(out=None), -1),
+    (dict(out=FAKE), -1),                      # out aliases q
+    (dict(B=0), -1), (dict(H=-1), -1), (dict(L_src=0), -1), (dict(L_ctx=-64), -1),
+    (dict(a_s=float("nan")), -1), (dict(a_f=1.5), -1), (dict(a_s=-0.1), -1),
+    (dict(D=96), -3), (dict(b=32), -3), (dict(dt=7), -3), (dict(dt=1, D=128), -3),
+    (dict(L_src=100), -2), (dict(L_ctx=96), -2),
+    (dict(L_src=65536 * 2, L_ctx=64, b=64), -3),  # N / b above 2048
+    (dict(B=70000, H=1), -3),
+    (dict(), -4),                                  # no workspace
+    (dict(ws=FAKE + (3 << 32), ws_bytes=16), -4),  # workspace too small
+])
+def test_argument_errors(L, kw, code):
+    assert _fwd(L, **kw) == code
+    assert isa.last_error() != ""
+
+
+def test_plan_and_sizes_errors(L):
+    assert L.isa_workspace_bytes(1, 1, 100, 64, 64, 64, 0.5, 0) == 0
+    assert "multiples" in isa.last_error()
+    with pytest.raises(isa.IsaError) as e:
+        isa.plan(1, 1, 64, 64, 80, 64, 0.5, 0.5)
+    assert e.value.code == -3
+
+
+def test_workspace_grows_with_size(L):
+    a = isa.workspace_bytes(1, 2, 512, 512, 64, 64, 0.5, isa.ISA_F32)
+    b = isa.workspace_bytes(1, 40, 16384, 16384, 128, 128, 0.25)
+    assert 0 < a < b
+    assert a % 256 == 0 and b % 256 == 0
+
+
+def test_launch_count(L):
+    assert isa.launch_count(1, 40, 16384, 16384, 128, 128, 0.25, 0.6) == 4
+    assert isa.launch_count(1, 40, 16384, 16384, 128, 128, 0.0, 0.6) == 3  # nothing to gather
+    assert isa.launch_count(1, 40, 100, 64, 128, 64, 0.25, 0.6) == 0
+
+
+def test_host_entry_rejects_before_copying(L):
+    assert L.isa_forward_host(None, FAKE, FAKE, 1, 1, 64, 64, 64, 64, 0.5, 0.5, 0, FAKE + 4096, None, None) == -1
+    assert L.isa_forward_host(FAKE, FAKE, FAKE, 1, 1, 64, 60, 64, 64, 0.5, 0.5, 0, FAKE + (1 << 30), None, None) == -2
