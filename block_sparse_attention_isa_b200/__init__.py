@@ -58,6 +58,7 @@ EXPORTS = (
     "isa_launch_count",
     "isa_selftest_wait_timeout",
     "isa_set_stage_events",
+    "isa_select_context_noalloc",
     "isa_last_error",
 )
 
@@ -109,6 +110,8 @@ def lib() -> ctypes.CDLL:
     L.isa_selftest_wait_timeout.restype = c_int
     L.isa_set_stage_events.argtypes = [vp, c_int]
     L.isa_set_stage_events.restype = c_int
+    L.isa_select_context_noalloc.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_int, vp, vp, vp]
+    L.isa_select_context_noalloc.restype = c_int
     L.isa_last_error.argtypes = []
     L.isa_last_error.restype = ctypes.c_char_p
     _LIB = L

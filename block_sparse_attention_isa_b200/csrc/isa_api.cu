@@ -94,6 +94,18 @@ bool overlaps(const void* a, const void* b, size_t bytes) {
 
 }  // namespace
 
+int build_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, int dt, Plan* p) {
+  return make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dt, p);
+}
+
+int set_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
 size_t workspace_layout(const Plan& p, Work* w, char* base) {
   size_t off = 0;
   auto take = [&](size_t bytes) -> char* {

@@ -55,6 +55,12 @@ enum : uint32_t {
 
 size_t workspace_layout(const Plan& p, Work* w, char* base);
 
+// Argument checks and block counts shared by the entry points (same rules and
+// messages as isa_forward_ex); returns ISA_OK or an error code.
+int build_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, int dt, Plan* p);
+// Sets the thread-local message returned by isa_last_error() and returns `code`.
+int set_error(int code, const char* fmt, ...);
+
 cudaError_t launch_pool_score_topk(const void* q, const void* k, const void* v, const Plan& p, const Work& w,
                                    cudaStream_t s);
 cudaError_t launch_gather(const void* k, const void* v, const Plan& p, const Work& w, cudaStream_t s);

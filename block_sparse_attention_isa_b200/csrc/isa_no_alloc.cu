@@ -1,0 +1,91 @@
+// Allocation-free entry point: the pooling + coarse-score + context top-k
+// kernel with its scratch memory in a fixed device array instead of a
+// caller-provided workspace.
+//
+// Why: some callers cannot allocate device memory. Plugin hosts of inference
+// runtimes often hand an operator only its input and output buffers and keep
+// every other byte of device memory to themselves, and latency-critical serving
+// loops may forbid cudaMalloc because it can synchronise the device. Such
+// callers can still ask which context blocks the pass would keep.
+//
+// How: the block means of Q, K and V and the per-head completion counters live
+// in `g_scratch`, a file-scope __device__ array of kScratchBytes. Every GPU that
+// loads this library holds that array until the process exits. Host code must
+// not pass the symbol itself to a kernel (on the host it names a host-side
+// stand-in); the device address is looked up once per device with
+// cudaGetSymbolAddress and cached.
+#include <mutex>
+
+#include "../../include/isa.h"
+#include "isa_internal.h"
+
+namespace isa {
+namespace {
+
+constexpr size_t kScratchBytes = size_t(32) << 20;  // 32 MiB per device
+__device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mutex;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Device address of g_scratch on the current device (looked up on first use).
+int scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return set_error(ISA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_scratch);
+    if (e != cudaSuccess || !ptr)
+      return set_error(ISA_ERR_CUDA, "cudaGetSymbolAddress of the fixed scratch array: %s", cudaGetErrorString(e));
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return ISA_OK;
+}
+
+}  // namespace
+}  // namespace isa
+
+using namespace isa;
+
+extern "C" int isa_select_context_noalloc(const void* q, const void* k, const void* v, int B, int H, int L_src,
+                                          int L_ctx, int D, int b, float alpha_s, isa_dtype dt, int32_t* sel,
+                                          float* colscore, void* stream) {
+  Plan p;
+  int rc = build_plan(B, H, L_src, L_ctx, D, b, alpha_s, 0.0f, (int)dt, &p);
+  if (rc != ISA_OK) return rc;
+  if (!q || !k || !v) return set_error(ISA_ERR_ARG, "q, k and v must not be NULL");
+  if (!sel || !colscore) return set_error(ISA_ERR_ARG, "sel and colscore must not be NULL");
+  const size_t BH = (size_t)p.BH;
+  const size_t ctr_bytes = align256(sizeof(uint32_t) * BH);
+  const size_t pooled_bytes = align256(sizeof(float) * BH * p.n_q * p.D);
+  const size_t need = ctr_bytes + 3 * pooled_bytes;
+  if (need > kScratchBytes)
+    return set_error(ISA_ERR_UNSUPPORTED,
+                     "these sizes need %zu bytes of scratch; the fixed array of the allocation-free entry point "
+                     "holds %zu (3 * B*H * (N/b) * D * 4 bytes plus counters must fit)",
+                     need, kScratchBytes);
+  void* base = nullptr;
+  if ((rc = scratch_address(&base)) != ISA_OK) return rc;
+  char* c = static_cast<char*>(base);
+  Work w{};
+  w.ctr_pool = reinterpret_cast<uint32_t*>(c);
+  w.qc = reinterpret_cast<float*>(c + ctr_bytes);
+  w.kc = reinterpret_cast<float*>(c + ctr_bytes + pooled_bytes);
+  w.vc = reinterpret_cast<float*>(c + ctr_bytes + 2 * pooled_bytes);
+  w.colscore = colscore;
+  w.sel = sel;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the array keeps the previous call's contents: the per-head counters must start at zero
+  cudaError_t e = cudaMemsetAsync(w.ctr_pool, 0, sizeof(uint32_t) * BH, s);
+  if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "clearing the scratch counters: %s", cudaGetErrorString(e));
+  e = launch_pool_score_topk(q, k, v, p, w, s);
+  if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "pool/score/top-k launch: %s", cudaGetErrorString(e));
+  return ISA_OK;
+}

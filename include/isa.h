@@ -162,6 +162,30 @@ ISA_API int isa_selftest_wait_timeout(void* workspace, int timeout_ms, void* str
  */
 ISA_API int isa_set_stage_events(void* const* events, int n_events);
 
+/*
+ * isa_select_context_noalloc - allocation-free form of stages 1-2 (pooling,
+ * coarse scores, context top-k). The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory, such as
+ * operator plugins that a host runtime hands only their input and output
+ * buffers, or serving loops that forbid cudaMalloc because it can
+ * synchronise the device.
+ *   q, k, v    device inputs [B, H, N, D] (as for isa_forward_ex)
+ *   sel        device int32 [B, H, k] output: kept context blocks, ascending
+ *   colscore   device float32 [B, H, N_ctx / b] output: context-block scores
+ * Scratch (the block means of Q, K, V and per-head counters,
+ * 3 * B*H * (N/b) * D * 4 bytes plus 4 bytes per head, each part rounded up
+ * to 256 bytes) lives in a fixed 32 MiB device array inside the library, which
+ * every GPU that loads the library holds until the process exits. Larger sizes
+ * return ISA_ERR_UNSUPPORTED before any GPU work. The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress); make that first
+ * call before any stream capture. Every call shares the one array: calls whose
+ * GPU work may overlap (several streams or host threads on one device) race on
+ * it and must be serialised by the caller. No allocation is made.
+ */
+ISA_API int isa_select_context_noalloc(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx,
+                                       int D, int b, float alpha_s, isa_dtype dt, int32_t* sel, float* colscore,
+                                       void* stream);
+
 /* Number of kernel launches one isa_forward_ex call makes for these sizes (0 if invalid). */
 ISA_API int isa_launch_count(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, isa_dtype dt);
 
