@@ -57,6 +57,7 @@ EXPORTS = (
     "isa_debug_pooled",
     "isa_launch_count",
     "isa_selftest_wait_timeout",
+    "isa_selftest_exp2",
     "isa_set_stage_events",
     "isa_select_context_noalloc",
     "isa_last_error",
@@ -108,6 +109,8 @@ def lib() -> ctypes.CDLL:
     L.isa_launch_count.restype = c_int
     L.isa_selftest_wait_timeout.argtypes = [vp, c_int, vp]
     L.isa_selftest_wait_timeout.restype = c_int
+    L.isa_selftest_exp2.argtypes = [vp, vp, vp, c_int, vp]
+    L.isa_selftest_exp2.restype = c_int
     L.isa_set_stage_events.argtypes = [vp, c_int]
     L.isa_set_stage_events.restype = c_int
     L.isa_select_context_noalloc.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_int, vp, vp, vp]

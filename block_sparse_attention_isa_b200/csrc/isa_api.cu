@@ -124,6 +124,7 @@ size_t workspace_layout(const Plan& p, Work* w, char* base) {
   t.kc = reinterpret_cast<float*>(take(sizeof(float) * BH * p.n_q * p.D));
   t.vc = reinterpret_cast<float*>(take(sizeof(float) * BH * p.n_q * p.D));
   t.colscore = reinterpret_cast<float*>(take(sizeof(float) * BH * p.n_ctx));
+  t.partial = reinterpret_cast<float*>(take(sizeof(float) * pool_partial_floats(p)));
   t.sel = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * BH * (p.k > 0 ? p.k : 1)));
   t.sharp = reinterpret_cast<float*>(take(sizeof(float) * BH * p.n_q));
   t.route = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * BH * p.n_q));
@@ -131,6 +132,10 @@ size_t workspace_layout(const Plan& p, Work* w, char* base) {
   t.vcn = take((size_t)p.elem * BH * p.n_new * p.D);
   t.ksel = take((size_t)p.elem * BH * (p.k > 0 ? p.k : 1) * p.b * p.D);
   t.vsel = take((size_t)p.elem * BH * (p.k > 0 ? p.k : 1) * p.b * p.D);
+  if (p.dt == ISA_F32) {
+    t.vtn = reinterpret_cast<float*>(take(sizeof(float) * BH * p.D * p.L_new));
+    t.vct = reinterpret_cast<float*>(take(sizeof(float) * BH * p.D * vct_ld(p)));
+  }
   if (w) *w = t;
   return off;
 }
@@ -176,6 +181,7 @@ int run_forward(const void* q, const void* k, const void* v, const Plan& p, void
   if ((e = launch_gather(k, v, p, w, s)) != cudaSuccess) return cuda_fail(e, "gather launch");
   if ((e = mark(2, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
   if ((e = launch_route(p, w, s)) != cudaSuccess) return cuda_fail(e, "routing launch");
+  if ((e = launch_transpose_v(v, p, w, s)) != cudaSuccess) return cuda_fail(e, "V transpose launch");
   if ((e = mark(3, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
   if ((e = launch_attention(q, k, v, out, p, w, s, nullptr)) != cudaSuccess) return cuda_fail(e, "attention launch");
   if ((e = mark(4, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
@@ -240,7 +246,7 @@ size_t isa_workspace_bytes(int B, int H, int L_src, int L_ctx, int D, int b, flo
 int isa_launch_count(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, isa_dtype dt) {
   Plan p;
   if (make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p) != ISA_OK) return 0;
-  return 3 + (p.k > 0 ? 1 : 0);
+  return 3 + (p.k > 0 ? 1 : 0) + (p.dt == ISA_F32 ? 1 : 0);
 }
 
 int isa_forward_ex(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
@@ -335,6 +341,13 @@ int isa_selftest_wait_timeout(void* workspace, int timeout_ms, void* stream) {
   if (timeout_ms <= 0 || timeout_ms > 10000) return fail(ISA_ERR_ARG, "timeout_ms must lie in [1, 10000]");
   cudaError_t e = launch_wait_selftest(static_cast<uint32_t*>(workspace), timeout_ms, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return ISA_OK;
+}
+
+int isa_selftest_exp2(const float* x, float* y_poly, float* y_ref, int n, void* stream) {
+  if (!x || !y_poly || !y_ref || n < 0) return fail(ISA_ERR_ARG, "x, y_poly and y_ref must not be NULL");
+  cudaError_t e = launch_exp2_selftest(x, y_poly, y_ref, n, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "exp2 self-test launch");
   return ISA_OK;
 }
 

@@ -22,15 +22,20 @@ struct Plan {
   int elem;    // bytes per element
 };
 
+// Row length of the transposed pooled V rows (fp32 inputs): n_new rounded up to 4
+// floats so that the rows start on 16-byte boundaries, as TMA requires.
+__host__ __device__ inline int vct_ld(const Plan& p) { return (p.n_new + 3) & ~3; }
+
 // Views into the caller's workspace (all 256-byte aligned).
 struct Work {
   uint32_t* ctrl;        // [kCtrlWords]: error word, spare words
-  uint32_t* ctr_pool;    // [BH] CTAs of the pooling grid finished per head
+  uint32_t* ctr_pool;    // [BH] scoring items finished per head (pooling kernel)
   uint32_t* ctr_route;   // [BH] CTAs of the routing grid finished per head
   float* qc;             // [BH, n_q, D] block means of Q (fp32)
   float* kc;             // [BH, n_q, D]
   float* vc;             // [BH, n_q, D]
   float* colscore;       // [BH, n_ctx] context-block scores
+  float* partial;        // [BH, ceil(n_src/16), n_ctx] per-item context-column sums (pooling kernel)
   int32_t* sel;          // [BH, max(k,1)] kept context blocks, ascending
   float* sharp;          // [BH, n_q] query-block sharpness M_i
   int32_t* route;        // [BH, n_q] exact blocks ascending, then Taylor blocks ascending
@@ -38,6 +43,8 @@ struct Work {
   void* vcn;             // [BH, n_new, D]
   void* ksel;            // [BH, k*b, D] gathered context keys
   void* vsel;            // [BH, k*b, D]
+  float* vtn;            // fp32 inputs only: [BH, D, L_new] V_new transposed
+  float* vct;            // fp32 inputs only: [BH, D, vct_ld] pooled V_new rows transposed
 };
 
 constexpr int kCtrlWords = 64;
@@ -51,7 +58,14 @@ enum : uint32_t {
   kErrSoftmax = 1u << 2,
   kErrGather = 1u << 3,
   kErrSelftest = 1u << 4,
+  kErrPool = 1u << 5,
 };
+
+// Control words at the start of the workspace (cleared on every call).
+enum : int { kCtrlError = 0, kCtrlGridBarrier = 1 };
+
+// Floats of the pooling kernel's per-item partial sums for these sizes.
+size_t pool_partial_floats(const Plan& p);
 
 size_t workspace_layout(const Plan& p, Work* w, char* base);
 
@@ -65,12 +79,15 @@ cudaError_t launch_pool_score_topk(const void* q, const void* k, const void* v, 
                                    cudaStream_t s);
 cudaError_t launch_gather(const void* k, const void* v, const Plan& p, const Work& w, cudaStream_t s);
 cudaError_t launch_route(const Plan& p, const Work& w, cudaStream_t s);
+cudaError_t launch_transpose_v(const void* v, const Plan& p, const Work& w, cudaStream_t s);
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out, const Plan& p,
                              const Work& w, cudaStream_t s, int* n_ctas_out);
 
 // One thread waits on an mbarrier that nothing arrives on; the bounded wait gives
 // up after `timeout_ms` and sets kErrSelftest in err[0].
 cudaError_t launch_wait_selftest(uint32_t* err, int timeout_ms, cudaStream_t s);
+// y_poly[i] = the attention softmax's polynomial 2^x[i]; y_ref[i] = CUDA's exp2f(x[i]).
+cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t s);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

@@ -8,8 +8,9 @@
 // loops may forbid cudaMalloc because it can synchronise the device. Such
 // callers can still ask which context blocks the pass would keep.
 //
-// How: the block means of Q, K and V and the per-head completion counters live
-// in `g_scratch`, a file-scope __device__ array of kScratchBytes. Every GPU that
+// How: the block means of Q, K and V, the per-item partial sums, the control
+// words and the per-head completion counters live in `g_scratch`, a file-scope
+// __device__ array of kScratchBytes. Every GPU that
 // loads this library holds that array until the process exits. Host code must
 // not pass the symbol itself to a kernel (on the host it names a host-side
 // stand-in); the device address is looked up once per device with
@@ -63,9 +64,11 @@ extern "C" int isa_select_context_noalloc(const void* q, const void* k, const vo
   if (!q || !k || !v) return set_error(ISA_ERR_ARG, "q, k and v must not be NULL");
   if (!sel || !colscore) return set_error(ISA_ERR_ARG, "sel and colscore must not be NULL");
   const size_t BH = (size_t)p.BH;
+  const size_t ctrl_bytes = align256(sizeof(uint32_t) * kCtrlWords);
   const size_t ctr_bytes = align256(sizeof(uint32_t) * BH);
   const size_t pooled_bytes = align256(sizeof(float) * BH * p.n_q * p.D);
-  const size_t need = ctr_bytes + 3 * pooled_bytes;
+  const size_t partial_bytes = align256(sizeof(float) * pool_partial_floats(p));
+  const size_t need = ctrl_bytes + ctr_bytes + 3 * pooled_bytes + partial_bytes;
   if (need > kScratchBytes)
     return set_error(ISA_ERR_UNSUPPORTED,
                      "these sizes need %zu bytes of scratch; the fixed array of the allocation-free entry point "
@@ -75,15 +78,18 @@ extern "C" int isa_select_context_noalloc(const void* q, const void* k, const vo
   if ((rc = scratch_address(&base)) != ISA_OK) return rc;
   char* c = static_cast<char*>(base);
   Work w{};
-  w.ctr_pool = reinterpret_cast<uint32_t*>(c);
-  w.qc = reinterpret_cast<float*>(c + ctr_bytes);
-  w.kc = reinterpret_cast<float*>(c + ctr_bytes + pooled_bytes);
-  w.vc = reinterpret_cast<float*>(c + ctr_bytes + 2 * pooled_bytes);
+  w.ctrl = reinterpret_cast<uint32_t*>(c);
+  w.ctr_pool = reinterpret_cast<uint32_t*>(c + ctrl_bytes);
+  w.qc = reinterpret_cast<float*>(c + ctrl_bytes + ctr_bytes);
+  w.kc = reinterpret_cast<float*>(c + ctrl_bytes + ctr_bytes + pooled_bytes);
+  w.vc = reinterpret_cast<float*>(c + ctrl_bytes + ctr_bytes + 2 * pooled_bytes);
+  w.partial = reinterpret_cast<float*>(c + ctrl_bytes + ctr_bytes + 3 * pooled_bytes);
   w.colscore = colscore;
   w.sel = sel;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the array keeps the previous call's contents: the per-head counters must start at zero
-  cudaError_t e = cudaMemsetAsync(w.ctr_pool, 0, sizeof(uint32_t) * BH, s);
+  // the array keeps the previous call's contents: the control words (error word,
+  // grid barrier) and the per-head counters must start at zero
+  cudaError_t e = cudaMemsetAsync(c, 0, ctrl_bytes + ctr_bytes, s);
   if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "clearing the scratch counters: %s", cudaGetErrorString(e));
   e = launch_pool_score_topk(q, k, v, p, w, s);
   if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "pool/score/top-k launch: %s", cudaGetErrorString(e));

@@ -17,11 +17,14 @@
 //    block takes exactly one path, so there is nothing to merge).
 //
 // Design for sm_100a (prior art on the pages is Triton / TileLang on Hopper):
-//  * one CTA per SM (persistent), 12 warps: warp 0 issues TMA loads, warp 1
+//  * one CTA per SM (persistent), 20 warps: warp 0 issues TMA loads, warp 1
 //    owns TMEM and issues tcgen05.mma from one thread (warps 2-3 idle), warps
-//    4-7 and 8-11 are two softmax warpgroups, one per 128-row query tile;
-//    each softmax thread owns one query row and keeps its 128 scores in
-//    registers (setmaxnreg moves registers from warpgroup 0 to them);
+//    4-19 are four softmax warpgroups, two per 128-row query tile: a query row
+//    is shared by two threads, each holding 64 of its 128 scores in registers
+//    (setmaxnreg moves registers from warpgroup 0 to them). The two halves
+//    exchange their partial row maxima through shared memory once per K/V
+//    tile, keep separate partial row sums (added once at the end), and each
+//    rescales and writes its own half of the output columns;
 //  * a work item is up to two 128-row query tiles of one head (four blocks
 //    when b = 64), both walking the same K/V tiles, so every K/V tile is
 //    loaded once for 256 query rows;
@@ -37,25 +40,50 @@
 #include <cudaTypedefs.h>
 #include <float.h>
 
+#include "exp2_poly.cuh"
 #include "isa_internal.h"
 #include "ptx.cuh"
 
 namespace isa {
 namespace {
 
-constexpr int kThreads = 384;  // 3 warpgroups
-// Register budget: the kernel is compiled for 168 registers a thread at launch
-// (384 x 168 = 64512 of the SM's 65536). Warpgroup 0 (TMA + MMA warps) gives
-// registers back and the two softmax warpgroups take them:
-// 128 x 56 + 256 x 224 = 64512, the same total, so the increase never waits.
-// The launcher checks the compiled count before every launch.
-constexpr int kLaunchRegs = 168;
-constexpr int kLowRegs = 56;
-constexpr int kHighRegs = 224;
-static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
+// Threads per query row in the softmax (1: a thread holds all 128 scores of its
+// row; 2: two threads hold 64 each and exchange partial row maxima). One thread
+// per row measured faster (4.78 ms against 6.05 ms at the 32K-token workload).
+#ifndef ISA_ROW_SPLIT
+#define ISA_ROW_SPLIT 1
+#endif
+constexpr int kSplit = ISA_ROW_SPLIT;
+static_assert(kSplit == 1 || kSplit == 2, "one or two threads per row");
+constexpr int kThreads = 128 + 256 * kSplit;  // warpgroup 0 + kSplit softmax warpgroups per query tile
+// Register budget: the kernel is compiled for kLaunchRegs registers a thread at
+// launch (kThreads x kLaunchRegs <= 65536). Warpgroup 0 (TMA + MMA warps) gives
+// registers back and the softmax warpgroups take them; the two shares add up to
+// at most the launch total, so the increase never waits. The launcher checks the
+// compiled count before every launch.
+constexpr int kLaunchRegs = kSplit == 1 ? 168 : 96;
+constexpr int kLowRegs = kSplit == 1 ? 88 : 64;
+constexpr int kHighRegs = kSplit == 1 ? 208 : 104;
+static_assert(128 * kLowRegs + 256 * kSplit * kHighRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch budget");
+constexpr int kCols = 128 / kSplit;  // scores per softmax thread
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per K/V tile
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain
+// Share of the exponentials computed by the FMA-pipe polynomial instead of ex2:
+// pair i of a row goes to the polynomial when (i % kPolyDen) < kPolyNum. On B200
+// the softmax is bound by instruction issue, not by the ex2 unit, so the
+// polynomial's extra instructions cost more than they save: measured at the
+// 32K-token workload, the attention kernel takes 4.78 ms with no polynomial
+// share, 5.07 ms with 1/4 and 5.44 ms with 1/2. It stays available here.
+#ifndef ISA_POLY_NUM
+#define ISA_POLY_NUM 0
+#endif
+#ifndef ISA_POLY_DEN
+#define ISA_POLY_DEN 4
+#endif
+constexpr int kPolyNum = ISA_POLY_NUM;
+constexpr int kPolyDen = ISA_POLY_DEN;
 
 struct AttnParams {
   const int32_t* route;
@@ -68,6 +96,18 @@ struct AttnParams {
   int items_t;   // Taylor items per head
   int total;     // all items
   float scale_log2;
+};
+
+struct Bars {
+  uint64_t q_full[2];
+  uint64_t q_empty;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], p_ready[2], o_done[2];
+  uint64_t drain;
+  uint64_t xbar[2];          // per query tile: both column halves (256 threads) have written their partial
+  uint32_t tmem_base;
+  int abort_flag;
+  float xpart[2][2][2][128];  // [exchange parity][query tile][column half][row]: partial row max or row sum
 };
 
 template <typename T, int D>
@@ -85,12 +125,16 @@ struct Cfg {
   static constexpr int STAGES = 2;
   static constexpr uint32_t FMT = kTf32 ? 2u : 1u;
   static constexpr uint32_t IDESC_QK = umma_idesc(FMT, kBM, kBN, 0, 0);
-  static constexpr uint32_t IDESC_PV = umma_idesc(FMT, kBM, D, 0, 1);
+  // bf16: V tiles as stored ([keys][D], MN-major B). tf32 takes B K-major only,
+  // so fp32 inputs load tiles of V^T ([D][keys], 32-key chunks of 128 bytes).
+  static constexpr bool kVT = kTf32;
+  static constexpr int VT_CH_STRIDE = D * 128;  // bytes between 32-key chunks of a V^T tile
+  static constexpr uint32_t IDESC_PV = umma_idesc(FMT, kBM, D, 0, kVT ? 0u : 1u);
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = 2 * TILE;
   static constexpr int OFF_V = OFF_K + STAGES * TILE;
   static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
-  static constexpr int SMEM_USED = OFF_BAR + 256;
+  static constexpr int SMEM_USED = OFF_BAR + (int)sizeof(Bars);
   // padded above half of the SM's shared memory so that exactly one CTA (and one
   // 512-column TMEM allocation) lives on each SM
   static constexpr int SMEM_ALLOC = (SMEM_USED + 1024 > 120 * 1024 ? SMEM_USED + 1024 : 120 * 1024);
@@ -135,15 +179,6 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p, int g) {
   return it;
 }
 
-struct Bars {
-  uint64_t q_full[2];
-  uint64_t q_empty;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], p_ready[2], o_done[2];
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort_flag;
-};
 
 __device__ __forceinline__ bool aborted(const Bars* b) {
   return *reinterpret_cast<const volatile int*>(&b->abort_flag) != 0;
@@ -204,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->q_full[t], 1);
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_ready[t], 128);
+      mbar_init(&bars->p_ready[t], 128 * kSplit);
       mbar_init(&bars->o_done[t], 1);
     }
     mbar_init(&bars->q_empty, 1);
@@ -215,6 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->v_empty[s], 1);
     }
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->xbar[0], 128 * kSplit);
+    mbar_init(&bars->xbar[1], 128 * kSplit);
     bars->abort_flag = 0;
     mbar_fence_init();
   }
@@ -234,16 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
 
   if (warp < 4) regs_dealloc<kLowRegs>();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t kv_it = 0, n_local = 0;
-      uint32_t q_arm[2] = {0, 0};
-      uint32_t k_arm[C::STAGES] = {}, v_arm[C::STAGES] = {};
+      uint32_t kv_it = 0, n_local = 0, k_issued = 0, v_issued = 0, q_arm0 = 0, q_arm1 = 0;
       bool ok = true;
       for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x, ++n_local) {
         const Item it = decode_item(p, g);
@@ -254,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int t = 0; t < it.ntiles; ++t) {
           mbar_arrive_expect_tx(&bars->q_full[t], C::TILE);
-          ++q_arm[t];
+          if (t == 0) ++q_arm0; else ++q_arm1;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int r = 64 * h;
@@ -274,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // K tile
           if (!mbar_wait(&bars->k_empty[st], ph ^ 1)) { raise_abort(bars, p.err, kErrProducer); ok = false; break; }
           mbar_arrive_expect_tx(&bars->k_full[st], C::TILE);
-          ++k_arm[st];
+          ++k_issued;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int r0 = j * kBN + 64 * h;
@@ -293,31 +327,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           // V tile
           if (!mbar_wait(&bars->v_empty[st], ph ^ 1)) { raise_abort(bars, p.err, kErrProducer); ok = false; break; }
           mbar_arrive_expect_tx(&bars->v_full[st], C::TILE);
-          ++v_arm[st];
+          ++v_issued;
+          if constexpr (C::kVT) {
+            // V^T tile: 4 chunks of 32 keys x D rows (tm_v / tm_vcn hold V_new^T / Vc_new^T here)
+            const CUtensorMap* map = it.kind == 0 ? &tm_v : &tm_vcn;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int r0 = j * kBN + 64 * h;
-            const CUtensorMap* map;
-            int y;
-            if (it.kind == 0) {
-              if (r0 < p.L_src) { map = &tm_v; y = r0; } else { map = &tm_vsel; y = r0 - p.L_src; }
-            } else {
-              map = &tm_vcn; y = r0;
+            for (int c = 0; c < 4; ++c)
+              tma_load_3d(sV + st * C::TILE + c * C::VT_CH_STRIDE, map, &bars->v_full[st], j * kBN + 32 * c, 0,
+                          it.bh);
+          } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int r0 = j * kBN + 64 * h;
+              const CUtensorMap* map;
+              int y;
+              if (it.kind == 0) {
+                if (r0 < p.L_src) { map = &tm_v; y = r0; } else { map = &tm_vsel; y = r0 - p.L_src; }
+              } else {
+                map = &tm_vcn; y = r0;
+              }
+#pragma unroll
+              for (int c = 0; c < C::NCH; ++c)
+                tma_load_3d(sV + st * C::TILE + c * C::CH_STRIDE + h * 8192, map, &bars->v_full[st],
+                            c * C::BOX_X, y, it.bh);
             }
-#pragma unroll
-            for (int c = 0; c < C::NCH; ++c)
-              tma_load_3d(sV + st * C::TILE + c * C::CH_STRIDE + h * 8192, map, &bars->v_full[st], c * C::BOX_X,
-                          y, it.bh);
           }
         }
       }
       if (!ok) {
         // let every copy this thread started land before the CTA can leave
-        for (int t = 0; t < 2; ++t)
-          if (q_arm[t]) mbar_wait(&bars->q_full[t], (q_arm[t] - 1) & 1);
-        for (int s = 0; s < C::STAGES; ++s) {
-          if (k_arm[s]) mbar_wait(&bars->k_full[s], (k_arm[s] - 1) & 1);
-          if (v_arm[s]) mbar_wait(&bars->v_full[s], (v_arm[s] - 1) & 1);
+        if (q_arm0) mbar_wait(&bars->q_full[0], (q_arm0 - 1) & 1);
+        if (q_arm1) mbar_wait(&bars->q_full[1], (q_arm1 - 1) & 1);
+        for (uint32_t s = 0; s < (uint32_t)C::STAGES; ++s) {
+          // tiles issued into stage s so far: those with index = s (mod STAGES)
+          const uint32_t ka = k_issued > s ? (k_issued - s + C::STAGES - 1) / C::STAGES : 0;
+          const uint32_t va = v_issued > s ? (v_issued - s + C::STAGES - 1) / C::STAGES : 0;
+          if (ka) mbar_wait(&bars->k_full[s], (ka - 1) & 1);
+          if (va) mbar_wait(&bars->v_full[s], (va - 1) & 1);
         }
       }
     }
@@ -325,28 +371,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t kv_it = 0;
-      uint32_t q_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
+      const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
+      uint32_t kv_it = 0, q_cnt0 = 0, q_cnt1 = 0, pv_cnt0 = 0, pv_cnt1 = 0;
       bool ok = true;
-      const uint32_t sq = smem_addr(sQ), sk = smem_addr(sK), sv = smem_addr(sV);
-      auto issue_s = [&](int t, int st) {
-        const uint32_t d = tmem + t * 128;
-        const uint32_t qa = sq + t * C::TILE, ka = sk + st * C::TILE;
+      // descriptor low words of the operand bases; every K-step adds a compile-time offset
+      constexpr uint32_t HI = desc_hi_sw128(1024);
+      const uint32_t q_lo0 = desc_lo(smem_addr(sQ), 16), q_lo1 = desc_lo(smem_addr(sQ + C::TILE), 16);
+      const uint32_t k_lo0 = desc_lo(smem_addr(sK), 16), k_lo1 = desc_lo(smem_addr(sK + C::TILE), 16);
+      const uint32_t v_lbo = C::kVT ? 16u : (uint32_t)C::CH_STRIDE;
+      const uint32_t v_lo0 = desc_lo(smem_addr(sV), v_lbo), v_lo1 = desc_lo(smem_addr(sV + C::TILE), v_lbo);
+      const uint32_t t_s0 = tmem, t_s1 = tmem + 128, t_o0 = tmem + 256, t_o1 = tmem + 384;
+      auto issue_s = [&](uint32_t d, uint32_t qa, uint32_t ka) {
 #pragma unroll
         for (int s = 0; s < C::KS_QK; ++s) {
-          const uint32_t off = (s / 4) * C::CH_STRIDE + (s % 4) * 32;
-          umma_ss<C::kTf32>(d, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), C::IDESC_QK,
-                            s > 0 ? 1u : 0u);
+          constexpr uint32_t dummy = 0;
+          (void)dummy;
+          const uint32_t off = (uint32_t)(((s / 4) * C::CH_STRIDE + (s % 4) * 32) >> 4);
+          umma_ss_lo<C::kTf32>(d, qa + off, ka + off, HI, C::IDESC_QK, s > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int st, bool acc) {
-        const uint32_t d = tmem + 256 + t * 128;
-        const uint32_t pa = tmem + t * 128;
-        const uint32_t va = sv + st * C::TILE;
+      auto issue_pv = [&](uint32_t d, uint32_t pa, uint32_t va, uint32_t acc) {
 #pragma unroll
-        for (int s = 0; s < C::KS_PV; ++s)
-          umma_ts<C::kTf32>(d, pa + s * 8, smem_desc_sw128(va + s * C::PV_K * 128, C::CH_STRIDE, 1024), C::IDESC_PV,
-                            (acc || s > 0) ? 1u : 0u);
+        for (int s = 0; s < C::KS_PV; ++s) {
+          const uint32_t off = C::kVT ? (uint32_t)(((s / 4) * C::VT_CH_STRIDE + (s % 4) * 32) >> 4)
+                                      : (uint32_t)((s * C::PV_K * 128) >> 4);
+          umma_ts_lo<C::kTf32>(d, pa + s * 8, va + off, HI, C::IDESC_PV, (acc | (uint32_t)s) != 0 ? 1u : 0u);
+        }
       };
       auto wait_or_abort = [&](uint64_t* bar, uint32_t par) -> bool {
         if (aborted(bars)) { ok = false; return false; }
@@ -356,43 +406,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x) {
         const Item it = decode_item(p, g);
-        for (int t = 0; t < it.ntiles; ++t) {
-          if (!wait_or_abort(&bars->q_full[t], q_cnt[t] & 1)) break;
-          ++q_cnt[t];
+        const bool two = it.ntiles > 1;
+        if (!wait_or_abort(&bars->q_full[0], q_cnt0 & 1)) break;
+        ++q_cnt0;
+        if (two) {
+          if (!wait_or_abort(&bars->q_full[1], q_cnt1 & 1)) break;
+          ++q_cnt1;
         }
-        if (!ok) break;
         // S_t for the first K/V tile
         {
-          const int st = kv_it % C::STAGES;
+          const uint32_t st = kv_it % C::STAGES;
           if (!wait_or_abort(&bars->k_full[st], (kv_it / C::STAGES) & 1)) break;
-          for (int t = 0; t < it.ntiles; ++t) {
-            issue_s(t, st);
-            umma_commit(&bars->s_full[t]);
+          const uint32_t ka = st ? k_lo1 : k_lo0;
+          issue_s(t_s0, q_lo0, ka);
+          umma_commit(&bars->s_full[0]);
+          if (two) {
+            issue_s(t_s1, q_lo1, ka);
+            umma_commit(&bars->s_full[1]);
           }
           umma_commit(&bars->k_empty[st]);
           if (it.nkv == 1) umma_commit(&bars->q_empty);
         }
-        for (int j = 0; j < it.nkv && ok; ++j, ++kv_it) {
-          const int st = kv_it % C::STAGES;
+        for (int j = 0; j < it.nkv; ++j, ++kv_it) {
+          const uint32_t st = kv_it % C::STAGES;
           if (!wait_or_abort(&bars->v_full[st], (kv_it / C::STAGES) & 1)) break;
           const bool more = (j + 1 < it.nkv);
-          const int st1 = (kv_it + 1) % C::STAGES;
-          for (int t = 0; t < it.ntiles; ++t) {
-            if (!wait_or_abort(&bars->p_ready[t], pv_cnt[t] & 1)) break;
-            issue_pv(t, st, j > 0);
-            umma_commit(&bars->o_done[t]);
-            ++pv_cnt[t];
+          const uint32_t st1 = (kv_it + 1) % C::STAGES;
+          const uint32_t va = st ? v_lo1 : v_lo0;
+          const uint32_t ka1 = st1 ? k_lo1 : k_lo0;
+          const uint32_t acc = j > 0 ? 1u : 0u;
+          // tile 0: P0 V_j, then S0 of the next K/V tile
+          if (!wait_or_abort(&bars->p_ready[0], pv_cnt0 & 1)) break;
+          issue_pv(t_o0, t_s0, va, acc);
+          umma_commit(&bars->o_done[0]);
+          ++pv_cnt0;
+          if (more) {
+            if (!wait_or_abort(&bars->k_full[st1], ((kv_it + 1) / C::STAGES) & 1)) break;
+            issue_s(t_s0, q_lo0, ka1);
+            umma_commit(&bars->s_full[0]);
+          }
+          // tile 1
+          if (two) {
+            if (!wait_or_abort(&bars->p_ready[1], pv_cnt1 & 1)) break;
+            issue_pv(t_o1, t_s1, va, acc);
+            umma_commit(&bars->o_done[1]);
+            ++pv_cnt1;
             if (more) {
-              if (t == 0 && !wait_or_abort(&bars->k_full[st1], ((kv_it + 1) / C::STAGES) & 1)) break;
-              issue_s(t, st1);
-              umma_commit(&bars->s_full[t]);
-              if (t == it.ntiles - 1) {
-                umma_commit(&bars->k_empty[st1]);
-                if (j + 2 == it.nkv) umma_commit(&bars->q_empty);
-              }
+              issue_s(t_s1, q_lo1, ka1);
+              umma_commit(&bars->s_full[1]);
             }
           }
-          if (!ok) break;
+          if (more) {
+            umma_commit(&bars->k_empty[st1]);
+            if (j + 2 == it.nkv) umma_commit(&bars->q_empty);
+          }
           umma_commit(&bars->v_empty[st]);
         }
       }
@@ -404,15 +471,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
     regs_alloc<kHighRegs>();
-    const int t = (warp - 4) >> 2;           // query tile of this warpgroup
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
+    const int sw = warp - 4;
+    const int t = sw / (4 * kSplit);         // query tile
+    const int h = (sw >> 2) % kSplit;        // column part of the scores and of the output
     const int wl = warp & 3;                 // TMEM lane quarter
     const int row = wl * 32 + lane;          // row inside the 128-row tile
     const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
-    const uint32_t t_s = tmem + lane_off + t * 128;
-    const uint32_t t_o = tmem + lane_off + 256 + t * 128;
-    uint32_t s_cnt = 0, pv_cnt = 0;
+    const uint32_t t_s = tmem + lane_off + t * 128 + h * kCols;                               // this thread's scores
+    const uint32_t t_p = tmem + lane_off + t * 128 + h * (sizeof(T) == 2 ? kCols / 2 : kCols);  // its P
+    const uint32_t t_o = tmem + lane_off + 256 + t * 128 + h * (D / kSplit);                  // its O columns
+    uint32_t s_cnt = 0, pv_cnt = 0, x_cnt = 0;
     bool ok = true;
     T* out = static_cast<T*>(p.out);
+    // Partial-value exchange with the thread that holds the other half of the row:
+    // write, arrive on the tile's barrier (256 arrivals), wait (bounded), read the
+    // partner's value. Buffers alternate with the exchange count, so a value is only
+    // overwritten after the partner has passed the next exchange.
+    auto exchange = [&](float v, float& partner) -> bool {
+      const uint32_t par = x_cnt & 1;
+      bars->xpart[par][t][h][row] = v;
+      mbar_arrive(&bars->xbar[t]);
+      if (!warp_wait(bars, &bars->xbar[t], par, p.err)) return false;
+      partner = bars->xpart[par][t][h ^ 1][row];
+      ++x_cnt;
+      return true;
+    };
     for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x) {
       const Item it = decode_item(p, g);
       if (t >= it.ntiles) continue;
@@ -420,54 +504,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < it.nkv; ++j) {
         if (!warp_wait(bars, &bars->s_full[t], s_cnt & 1, p.err)) { ok = false; break; }
         ++s_cnt;
-        uint32_t r[128];
+        uint32_t r[kCols];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, r + 32 * c);
-        tmem_ld_wait<128>(r);
-        const int valid = (j == it.nkv - 1) ? it.last_valid : kBN;
-        float mx = -FLT_MAX;
+        for (int c = 0; c < kCols / 32; ++c) tmem_ld32(t_s + 32 * c, r + 32 * c);
+        tmem_ld_wait<kCols>(r);
+        if (j == it.nkv - 1 && it.last_valid < kBN) {  // ragged last K/V tile (uniform branch)
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          float x = __uint_as_float(r[i]) * p.scale_log2;
-          x = (i < valid) ? x : -FLT_MAX;
-          r[i] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+          for (int i = 0; i < kCols; ++i)
+            if (h * kCols + i >= it.last_valid) r[i] = __float_as_uint(-INFINITY);
         }
+        // (partial) row max of the raw scores: 4 independent chains of 3-input max
+        float mc[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mc[c] = __uint_as_float(r[c]);
+#pragma unroll
+        for (int i = 4; i < kCols; i += 8) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[i + c]), __uint_as_float(r[i + 4 + c]));
+        }
+        float pm = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+        if constexpr (kSplit == 2) {
+          // exchange with the thread holding the other half of the row (the exchange also
+          // guarantees that both halves have read their scores before P overwrites them)
+          float pm_other;
+          if (!exchange(pm, pm_other)) { ok = false; break; }
+          pm = fmaxf(pm, pm_other);
+        }
+        const float mx = pm * p.scale_log2;
         // lazy max: move it only when the tile's max exceeds it by more than 2^8
         const bool need = (j > 0) && (mx > m + kRescaleThreshold);
         const float alpha = need ? ex2_approx(m - mx) : 1.0f;
         if (j == 0 || need) m = mx;
-        float rs = 0.f;
-        if constexpr (sizeof(T) == 2) {
+        // p = 2^(s * scale - m), in pairs; one pair in kPolyEvery on the FMA pipe, the rest on ex2
+        const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(-m, -m);
+        uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const float p0 = ex2_approx(__uint_as_float(r[2 * i]) - m);
-            const float p1 = ex2_approx(__uint_as_float(r[2 * i + 1]) - m);
-            rs += p0 + p1;
-            __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-            r[i] = *reinterpret_cast<uint32_t*>(&h);
+        for (int i = 0; i < kCols / 2; ++i) {
+          const uint64_t x = ffma2(static_cast<uint64_t>(r[2 * i]) | (static_cast<uint64_t>(r[2 * i + 1]) << 32), sc2,
+                                   nm2);
+          uint64_t e;
+          if (i % kPolyDen < kPolyNum) e = exp2_poly2(x);
+          else e = pack2(ex2_approx(lo2(x)), ex2_approx(hi2(x)));
+          acc[i & 3] = fadd2(acc[i & 3], e);
+          if constexpr (sizeof(T) == 2) {
+            __nv_bfloat162 hv = __floats2bfloat162_rn(lo2(e), hi2(e));
+            r[i] = *reinterpret_cast<uint32_t*>(&hv);
+          } else {
+            r[2 * i] = static_cast<uint32_t>(e);
+            r[2 * i + 1] = static_cast<uint32_t>(e >> 32);
           }
-          tmem_st32(t_s, r);
-          tmem_st32(t_s + 32, r + 32);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 128; ++i) {
-            const float pv = ex2_approx(__uint_as_float(r[i]) - m);
-            rs += pv;
-            r[i] = __float_as_uint(pv);
-          }
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_st32(t_s + 32 * c, r + 32 * c);
         }
-        l = l * alpha + rs;
+#pragma unroll
+        for (int c = 0; c < (sizeof(T) == 2 ? kCols / 64 : kCols / 32); ++c) tmem_st32(t_p + 32 * c, r + 32 * c);
+        const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+        l = l * alpha + (lo2(a2) + hi2(a2));
         // O holds P V up to tile j-1; rows whose max moved are rescaled in place
-        // before P V of tile j may start. TMEM moves are warp-collective, so the
-        // whole warp takes this step when any of its rows needs it (alpha = 1 for
-        // the others).
+        // (this half's columns) before P V of tile j may start. TMEM moves are
+        // warp-collective, so the whole warp takes this step when any of its rows
+        // needs it (alpha = 1 for the others).
         if (__any_sync(0xffffffffu, need)) {
           if (!warp_wait(bars, &bars->o_done[t], (pv_cnt - 1) & 1, p.err)) { ok = false; break; }
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < D / 32 / kSplit; ++c) {
             uint32_t o[32];
             tmem_ld32(t_o + 32 * c, o);
             tmem_ld_wait<32>(o);
@@ -482,15 +580,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++pv_cnt;
       }
       if (!ok) break;
-      // epilogue: O / l written at the row's original token position
-      if (!warp_wait(bars, &bars->o_done[t], (pv_cnt - 1) & 1, p.err)) { ok = false; break; }
+      // epilogue: O / (l_half0 + l_half1) for this half's columns, at the row's original token position
+      if constexpr (kSplit == 2) {
+        float l_other;
+        if (!exchange(l, l_other)) { ok = false; break; }
+        l += l_other;
+      }
       const float inv_l = 1.0f / l;
+      if (!warp_wait(bars, &bars->o_done[t], (pv_cnt - 1) & 1, p.err)) { ok = false; break; }
       const int u = t * p.bpt + row / p.b;
       const bool store = (u < it.nblk);
       const size_t token = (size_t)it.blk(store ? u : 0) * p.b + (row % p.b);
-      T* dst = out + ((size_t)it.bh * p.N + token) * D;
+      T* dst = out + ((size_t)it.bh * p.N + token) * D + h * (D / kSplit);
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 32 / kSplit; ++c) {
         uint32_t o[32];
         tmem_ld32(t_o + 32 * c, o);
         tmem_ld_wait<32>(o);
@@ -507,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(*reinterpret_cast<volatile uint32_t*>(&bars->tmem_base), 512);
   }
 }
 
@@ -535,6 +638,21 @@ bool make_map(CUtensorMap* m, const void* base, int elem, int D, int rows, int h
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// fp32 [heads][D][keys] view of a transposed V, box of 32 keys x D rows, 128-byte swizzle,
+// keys past the end read as zeros.
+bool make_map_t(CUtensorMap* m, const void* base, int keys, int ld, int D, int heads) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)keys, (cuuint64_t)D, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 4, (cuuint64_t)ld * D * 4};
+  cuuint32_t box[3] = {32u, (cuuint32_t)D, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -567,12 +685,20 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, void* out, con
   const int E = sizeof(T);
   CUtensorMap tq, tk, tks, tv, tvs, tkc, tvc;
   const bool has_sel = pl.k > 0;
-  if (!make_map(&tq, q, E, D, pl.N, pl.BH) || !make_map(&tk, k, E, D, pl.N, pl.BH) ||
-      !make_map(&tv, v, E, D, pl.N, pl.BH) ||
-      !make_map(&tks, has_sel ? w.ksel : k, E, D, has_sel ? pl.k * pl.b : pl.N, pl.BH) ||
-      !make_map(&tvs, has_sel ? w.vsel : v, E, D, has_sel ? pl.k * pl.b : pl.N, pl.BH) ||
-      !make_map(&tkc, w.kcn, E, D, pl.n_new, pl.BH) || !make_map(&tvc, w.vcn, E, D, pl.n_new, pl.BH))
-    return cudaErrorInvalidValue;
+  bool ok = make_map(&tq, q, E, D, pl.N, pl.BH) && make_map(&tk, k, E, D, pl.N, pl.BH) &&
+            make_map(&tks, has_sel ? w.ksel : k, E, D, has_sel ? pl.k * pl.b : pl.N, pl.BH) &&
+            make_map(&tkc, w.kcn, E, D, pl.n_new, pl.BH);
+  if (C::kVT) {
+    // V_new^T [BH][D][L_new] and Vc_new^T [BH][D][n_new]: rows are D, the inner axis is the key
+    ok = ok && make_map_t(&tv, w.vtn, pl.L_new, pl.L_new, D, pl.BH) &&
+         make_map_t(&tvc, w.vct, pl.n_new, vct_ld(pl), D, pl.BH);
+    tvs = tv;
+  } else {
+    ok = ok && make_map(&tv, v, E, D, pl.N, pl.BH) &&
+         make_map(&tvs, has_sel ? w.vsel : v, E, D, has_sel ? pl.k * pl.b : pl.N, pl.BH) &&
+         make_map(&tvc, w.vcn, E, D, pl.n_new, pl.BH);
+  }
+  if (!ok) return cudaErrorInvalidValue;
 
   auto kern = attention_kernel<T, D>;
   cudaFuncAttributes fa;

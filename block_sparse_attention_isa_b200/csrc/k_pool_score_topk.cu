@@ -6,156 +6,213 @@
 // Method: "Lightning Unified Video Editing via In-Context Sparse Attention",
 // papernotes.org notes, Key design 1 (Context Pre-Selection), and the
 // paperlayer.ai summary, section 2 (Pooling Attention) and section 3
-// (Pre-Selection).
-//
-// Grid (n_q, B*H), 256 threads. Each CTA pools one block of b tokens of Q, K
-// and V with 16-byte vector loads (all loads of a thread issued before any
-// use, fp32 sums). The last CTA to finish a head (atomic counter after a
-// __threadfence) then scores that head:
+// (Pre-Selection):
+//   Qc, Kc, Vc = means over blocks of b tokens,
 //   S_coarse[i, :] = softmax_j(Qc_i . Kc_j / sqrt(D)) for source blocks i,
 //   score[c] = mean_i S_coarse[i, n_src + c],
 //   sel = the k largest scores (ties by lower index), stored ascending.
-// Work per head is n_src * n_q * D multiply-adds on the CUDA cores; the pooling
-// pass itself is bound by HBM (it reads Q, K and V once).
+//
+// One persistent cooperative launch, one CTA per SM, 256 threads:
+//  * phase 1 (HBM-bound): pooling units (head, block) are dealt round-robin to
+//    the CTAs; each unit's Q, K and V blocks (b contiguous rows each) arrive in
+//    a ring of shared-memory stages by 1-D TMA bulk copies, so several units
+//    are in flight per SM while the previous one is reduced (fp32 sums, 4-byte
+//    words, conflict-free shared-memory reads);
+//  * a grid barrier (all block means written);
+//  * phase 2: scoring items (head, 16 source rows) are dealt round-robin; each
+//    computes its rows of S_coarse (CUDA cores, fp32), their softmax, and the
+//    rows' sum on every context column, written as a partial. The last item of
+//    a head to finish adds the partials in a fixed order (deterministic), then
+//    runs the top-k as a shared-memory bitonic sort.
+// Every wait is bounded and reports through the error word.
 #include <cuda_bf16.h>
 #include <float.h>
 
 #include "block_sort.cuh"
 #include "isa_internal.h"
+#include "ptx.cuh"
 
 namespace isa {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kRowsPerChunk = 8;  // source query blocks scored per pass
+constexpr int kRows = 16;                  // source query blocks per scoring item
+constexpr int kStageBudget = 192 * 1024;   // shared memory for the phase-1 ring
+constexpr int kMaxStages = 8;
+
+template <typename T, int D, int BLK>
+struct PoolCfg {
+  static constexpr int E = sizeof(T);
+  static constexpr int TENSOR_BYTES = BLK * D * E;          // one block of one tensor
+  static constexpr int STAGE_BYTES = 3 * TENSOR_BYTES;
+  static constexpr int STAGES = (kStageBudget / STAGE_BYTES) < kMaxStages ? (kStageBudget / STAGE_BYTES) : kMaxStages;
+  static constexpr int WPR = D * E / 4;                     // 4-byte words per row
+  static constexpr int RG = kThreads / WPR;                 // row groups
+  static constexpr int FPW = 4 / E;                         // floats per word
+  static constexpr int RED_FLOATS = 3 * RG * D;             // phase-1 reduction scratch
+  static_assert(kThreads % WPR == 0 && BLK % RG == 0, "layout");
+  static_assert(STAGES >= 2, "at least two stages");
+};
+
+int score_scratch_floats(const Plan& p, int D) {
+  const int P = next_pow2(p.n_ctx < 1 ? 1 : p.n_ctx);
+  return kRows * D + kRows * p.n_q + p.n_ctx + 2 * P + next_pow2(p.k < 1 ? 1 : p.k);
+}
 
 template <typename T>
-struct Vec16;
+__device__ __forceinline__ void add_word(float* acc, uint32_t u);
 template <>
-struct Vec16<__nv_bfloat16> {
-  static constexpr int n = 8;
-  __device__ static void add(float* acc, const uint4& u) {
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(h[i]);
-      acc[2 * i] += f.x;
-      acc[2 * i + 1] += f.y;
-    }
-  }
-};
+__device__ __forceinline__ void add_word<__nv_bfloat16>(float* acc, uint32_t u) {
+  acc[0] += __uint_as_float(u << 16);
+  acc[1] += __uint_as_float(u & 0xffff0000u);
+}
 template <>
-struct Vec16<float> {
-  static constexpr int n = 4;
-  __device__ static void add(float* acc, const uint4& u) {
-    acc[0] += __uint_as_float(u.x);
-    acc[1] += __uint_as_float(u.y);
-    acc[2] += __uint_as_float(u.z);
-    acc[3] += __uint_as_float(u.w);
-  }
-};
+__device__ __forceinline__ void add_word<float>(float* acc, uint32_t u) {
+  acc[0] += __uint_as_float(u);
+}
 
-template <int D>
-size_t score_smem_bytes(const Plan& p) {
-  const int P = next_pow2(p.n_ctx < 1 ? 1 : p.n_ctx);
-  return sizeof(float) * (size_t)(kRowsPerChunk * D + kRowsPerChunk * p.n_q + p.n_ctx) +
-         (sizeof(float) + sizeof(int32_t)) * (size_t)P + sizeof(int32_t) * (size_t)next_pow2(p.k < 1 ? 1 : p.k);
+__device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t* err) {
+  __syncthreads();
+  __shared__ int s_ok;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(counter, 1u);
+    const uint64_t t0 = global_timer_ns();
+    int ok = 1;
+    while (true) {
+      uint32_t c;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(counter) : "memory");
+      if (c >= gridDim.x) break;
+      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        atomicOr(err, kErrPool);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
 }
 
 template <typename T, int D, int BLK>
-__global__ void __launch_bounds__(kThreads) pool_score_topk_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                                   const T* __restrict__ v, Plan p, Work w) {
-  extern __shared__ __align__(16) float smem[];
-  constexpr int VEC = Vec16<T>::n;
-  constexpr int TPR = D / VEC;           // threads per row
-  constexpr int RPP = kThreads / TPR;    // rows per pass
-  constexpr int PASSES = BLK / RPP;
-  static_assert(BLK % RPP == 0, "block size must be a multiple of the rows per pass");
+__global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                                      const T* __restrict__ v, Plan p, Work w) {
+  using C = PoolCfg<T, D, BLK>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  float* red = reinterpret_cast<float*>(full + kMaxStages);
+  const int tid = threadIdx.x, G = gridDim.x, g = blockIdx.x;
+  const int n_units = p.BH * p.n_q;
+  const T* src[3] = {q, k, v};
 
-  const int blk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-  const int col0 = (tid % TPR) * VEC, r0 = tid / TPR;
-  const size_t base = ((size_t)bh * p.N + (size_t)blk * BLK) * D + col0;
-
-  // ---- stage 1a: block means of Q, K, V ---------------------------------------------
-  float acc[3][VEC];
-#pragma unroll
-  for (int t = 0; t < 3; ++t)
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) acc[t][i] = 0.f;
-  {
-    uint4 buf[3][PASSES];
-#pragma unroll
-    for (int s = 0; s < PASSES; ++s) {
-      const size_t off = base + (size_t)(r0 + s * RPP) * D;
-      buf[0][s] = __ldcs(reinterpret_cast<const uint4*>(q + off));
-      buf[1][s] = __ldcs(reinterpret_cast<const uint4*>(k + off));
-      buf[2][s] = __ldcs(reinterpret_cast<const uint4*>(v + off));
-    }
-#pragma unroll
-    for (int s = 0; s < PASSES; ++s)
-#pragma unroll
-      for (int t = 0; t < 3; ++t) Vec16<T>::add(acc[t], buf[t][s]);
-  }
-  float* red = smem;  // [3][RPP][D]
-#pragma unroll
-  for (int t = 0; t < 3; ++t)
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) red[(t * RPP + r0) * D + col0 + i] = acc[t][i];
-  __syncthreads();
-  const float inv_b = 1.0f / (float)BLK;
-  for (int e = tid; e < 3 * D; e += kThreads) {
-    const int t = e / D, c = e % D;
-    float s = 0.f;
-#pragma unroll 4
-    for (int r = 0; r < RPP; ++r) s += red[(t * RPP + r) * D + c];
-    float* dst = (t == 0 ? w.qc : t == 1 ? w.kc : w.vc) + ((size_t)bh * p.n_q + blk) * D;
-    dst[c] = s * inv_b;
-  }
-
-  // ---- last CTA of this head scores it ----------------------------------------------
-  __shared__ int s_last;
-  __threadfence();  // make this thread's block means visible device-wide before the count
-  __syncthreads();
+  // ---- phase 1: block means --------------------------------------------------------
   if (tid == 0) {
-    const unsigned prev = atomicAdd(&w.ctr_pool[bh], 1u);
-    s_last = (prev == (unsigned)(p.n_q - 1));
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(&full[s], 1);
+    mbar_fence_init();
   }
   __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  auto issue = [&](int u, int s) {  // thread 0: the three blocks of unit u into stage s
+    const int bh = u / p.n_q, blk = u - bh * p.n_q;
+    const size_t off = ((size_t)bh * p.N + (size_t)blk * BLK) * D;
+    uint8_t* dst = smem + s * C::STAGE_BYTES;
+    mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+    for (int t = 0; t < 3; ++t) bulk_load(dst + t * C::TENSOR_BYTES, src[t] + off, C::TENSOR_BYTES, &full[s]);
+  };
+  const int my_units = g < n_units ? (n_units - g + G - 1) / G : 0;
+  int issued = 0;  // thread 0: units whose copies were started (unit i goes to stage i % STAGES)
+  if (tid == 0)
+    for (int i = 0; i < C::STAGES && i < my_units; ++i, ++issued) issue(g + i * G, i);
+  const int wd = tid % C::WPR, rg = tid / C::WPR;
+  bool ok = true;
+  for (int i = 0; i < my_units; ++i) {
+    const int s = i % C::STAGES, u = g + i * G;
+    const int bh = u / p.n_q, blk = u - bh * p.n_q;
+    int good = mbar_wait(&full[s], (i / C::STAGES) & 1) ? 1 : 0;
+    if (!__syncthreads_and(good)) {
+      if (tid == 0) atomicOr(&w.ctrl[kCtrlError], kErrPool);
+      ok = false;
+      break;
+    }
+    const uint32_t* base = reinterpret_cast<const uint32_t*>(smem + s * C::STAGE_BYTES);
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+      float acc[C::FPW];
+#pragma unroll
+      for (int f = 0; f < C::FPW; ++f) acc[f] = 0.f;
+      const uint32_t* tb = base + t * (C::TENSOR_BYTES / 4);
+#pragma unroll 8
+      for (int r = rg; r < BLK; r += C::RG) add_word<T>(acc, tb[r * C::WPR + wd]);
+#pragma unroll
+      for (int f = 0; f < C::FPW; ++f) red[(t * C::RG + rg) * D + wd * C::FPW + f] = acc[f];
+    }
+    __syncthreads();  // stage s fully read; partial sums in `red`
+    if (tid == 0 && i + C::STAGES < my_units) {
+      fence_proxy_async_smem();
+      issue(g + (i + C::STAGES) * G, s);
+      ++issued;
+    }
+    const float inv_b = 1.0f / (float)BLK;
+    for (int e = tid; e < 3 * D; e += kThreads) {
+      const int t = e / D, c = e - t * D;
+      float sum = 0.f;
+#pragma unroll
+      for (int r = 0; r < C::RG; ++r) sum += red[(t * C::RG + r) * D + c];
+      float* dst = (t == 0 ? w.qc : t == 1 ? w.kc : w.vc) + ((size_t)bh * p.n_q + blk) * D;
+      dst[c] = sum * inv_b;
+    }
+    __syncthreads();  // `red` free for the next unit
+  }
+  if (!ok) {
+    // let this CTA's outstanding copies land before leaving: wait for the last
+    // phase armed on every stage
+    if (tid == 0)
+      for (int st = 0; st < C::STAGES && st < issued; ++st) {
+        const int armed = (issued - st + C::STAGES - 1) / C::STAGES;
+        mbar_wait(&full[st], (armed - 1) & 1);
+      }
+    return;
+  }
 
+  // ---- grid barrier: every block mean is written --------------------------------------
+  if (!grid_barrier(&w.ctrl[kCtrlGridBarrier], &w.ctrl[kCtrlError])) return;
+
+  // ---- phase 2: coarse scores, context-column partial sums, top-k ----------------------
   const int n_q = p.n_q, n_src = p.n_src, n_ctx = p.n_ctx;
-  float* qcs = smem;                              // [R][D]
-  float* lg = qcs + kRowsPerChunk * D;            // [R][n_q]
-  float* cs = lg + kRowsPerChunk * n_q;           // [n_ctx]
+  const int n_chunks = (n_src + kRows - 1) / kRows;
+  float* qcs = reinterpret_cast<float*>(smem);      // [kRows][D]
+  float* lg = qcs + kRows * D;                      // [kRows][n_q]
+  float* cs = lg + kRows * n_q;                     // [n_ctx]
   const int P = next_pow2(n_ctx < 1 ? 1 : n_ctx);
-  float* skey = cs + n_ctx;                       // [P]
-  int32_t* sidx = reinterpret_cast<int32_t*>(skey + P);  // [P]
-  int32_t* ssel = sidx + P;                       // [next_pow2(k)]
-  const float* Qc = w.qc + (size_t)bh * n_q * D;
-  const float* Kc = w.kc + (size_t)bh * n_q * D;
+  float* skey = cs + n_ctx;                         // [P]
+  int32_t* sidx = reinterpret_cast<int32_t*>(skey + P);
+  int32_t* ssel = sidx + P;
   const float scale = 1.0f / sqrtf((float)D);
   const int lane = tid & 31, warp = tid >> 5;
-
-  for (int c = tid; c < n_ctx; c += kThreads) cs[c] = 0.f;
-  for (int i0 = 0; i0 < n_src; i0 += kRowsPerChunk) {
-    const int nr = min(kRowsPerChunk, n_src - i0);
+  __shared__ int s_last;
+  for (int item = g; item < p.BH * n_chunks; item += G) {
+    const int bh = item / n_chunks, chunk = item - bh * n_chunks;
+    const int i0 = chunk * kRows, nr = min(kRows, n_src - i0);
+    const float* Qc = w.qc + (size_t)bh * n_q * D;
+    const float* Kc = w.kc + (size_t)bh * n_q * D;
     __syncthreads();
-    for (int e = tid; e < kRowsPerChunk * D; e += kThreads) {
+    for (int e = tid; e < kRows * D; e += kThreads) {
       const int r = e / D;
-      qcs[e] = r < nr ? __ldcg(Qc + (size_t)(i0 + r) * D + (e % D)) : 0.f;
+      qcs[e] = r < nr ? __ldcg(Qc + (size_t)(i0 + r) * D + (e - r * D)) : 0.f;
     }
     __syncthreads();
     for (int j = tid; j < n_q; j += kThreads) {
-      float a[kRowsPerChunk];
+      float a[kRows];
 #pragma unroll
-      for (int r = 0; r < kRowsPerChunk; ++r) a[r] = 0.f;
+      for (int r = 0; r < kRows; ++r) a[r] = 0.f;
       const float4* kr = reinterpret_cast<const float4*>(Kc + (size_t)j * D);
-#pragma unroll 4
+#pragma unroll 2
       for (int d4 = 0; d4 < D / 4; ++d4) {
         const float4 kv = __ldcg(kr + d4);
 #pragma unroll
-        for (int r = 0; r < kRowsPerChunk; ++r) {
+        for (int r = 0; r < kRows; ++r) {
           const float4 qv = *reinterpret_cast<const float4*>(qcs + r * D + 4 * d4);
           a[r] = fmaf(qv.x, kv.x, a[r]);
           a[r] = fmaf(qv.y, kv.y, a[r]);
@@ -164,74 +221,92 @@ __global__ void __launch_bounds__(kThreads) pool_score_topk_kernel(const T* __re
         }
       }
 #pragma unroll
-      for (int r = 0; r < kRowsPerChunk; ++r)
+      for (int r = 0; r < kRows; ++r)
         if (r < nr) lg[r * n_q + j] = a[r] * scale;
     }
     __syncthreads();
-    // row softmax, one warp per row; only the context columns are kept
-    for (int r = warp; r < nr; r += kThreads / 32) {
+    for (int r = warp; r < nr; r += kThreads / 32) {  // row softmax, one warp per row
       float* row = lg + r * n_q;
       float m = -FLT_MAX;
       for (int j = lane; j < n_q; j += 32) m = fmaxf(m, row[j]);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      float s = 0.f;
-      for (int j = lane; j < n_q; j += 32) s += expf(row[j] - m);
+      float sum = 0.f;
+      for (int j = lane; j < n_q; j += 32) sum += expf(row[j] - m);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      const float inv = 1.0f / s;
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      const float inv = 1.0f / sum;
       __syncwarp();
       for (int c = lane; c < n_ctx; c += 32) row[n_src + c] = expf(row[n_src + c] - m) * inv;
     }
     __syncthreads();
+    float* part = w.partial + ((size_t)bh * n_chunks + chunk) * n_ctx;
     for (int c = tid; c < n_ctx; c += kThreads) {
-      float s = cs[c];
-      for (int r = 0; r < nr; ++r) s += lg[r * n_q + n_src + c];
-      cs[c] = s;
+      float sum = 0.f;
+      for (int r = 0; r < nr; ++r) sum += lg[r * n_q + n_src + c];
+      part[c] = sum;
     }
-  }
-  __syncthreads();
-  const float inv_src = 1.0f / (float)n_src;
-  for (int c = tid; c < P; c += kThreads) {
-    if (c < n_ctx) {
-      const float sc = cs[c] * inv_src;
-      w.colscore[(size_t)bh * n_ctx + c] = sc;
-      skey[c] = sc;
-      sidx[c] = c;
-    } else {
-      skey[c] = -FLT_MAX;
-      sidx[c] = 0x7fffffff - (c - n_ctx);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(&w.ctr_pool[bh], 1u) == (unsigned)(n_chunks - 1));
+    __syncthreads();
+    if (!s_last) continue;
+    __threadfence();
+    // this head is complete: context scores in a fixed order, then the top-k
+    const float inv_src = 1.0f / (float)n_src;
+    for (int c = tid; c < P; c += kThreads) {
+      if (c < n_ctx) {
+        float sum = 0.f;
+        for (int ch = 0; ch < n_chunks; ++ch) sum += __ldcg(w.partial + ((size_t)bh * n_chunks + ch) * n_ctx + c);
+        const float sc = sum * inv_src;
+        w.colscore[(size_t)bh * n_ctx + c] = sc;
+        skey[c] = sc;
+        sidx[c] = c;
+      } else {
+        skey[c] = -FLT_MAX;
+        sidx[c] = 0x7fffffff - (c - n_ctx);
+      }
     }
-  }
-  bitonic_sort_pairs<true>(skey, sidx, P);
-  // the k winners, re-sorted by block index
-  const int kk = p.k;
-  if (kk > 0) {
-    const int PK = next_pow2(kk);
-    for (int i = tid; i < PK; i += kThreads) ssel[i] = i < kk ? sidx[i] : 0x7fffffff;
-    bitonic_sort_int(ssel, PK);
-    for (int i = tid; i < kk; i += kThreads) w.sel[(size_t)bh * kk + i] = ssel[i];
+    bitonic_sort_pairs<true>(skey, sidx, P);
+    const int kk = p.k;
+    if (kk > 0) {
+      const int PK = next_pow2(kk);
+      for (int i = tid; i < PK; i += kThreads) ssel[i] = i < kk ? sidx[i] : 0x7fffffff;
+      bitonic_sort_int(ssel, PK);
+      for (int i = tid; i < kk; i += kThreads) w.sel[(size_t)bh * kk + i] = ssel[i];
+    }
   }
 }
 
 template <typename T, int D, int BLK>
 cudaError_t launch_t(const void* q, const void* k, const void* v, const Plan& p, const Work& w, cudaStream_t s) {
-  constexpr int VEC = 16 / sizeof(T);
-  constexpr int RPP = kThreads / (D / VEC);
-  const size_t pool_bytes = sizeof(float) * 3 * RPP * D;
-  const size_t smem = pool_bytes > score_smem_bytes<D>(p) ? pool_bytes : score_smem_bytes<D>(p);
+  using C = PoolCfg<T, D, BLK>;
+  const size_t ring = (size_t)C::STAGES * C::STAGE_BYTES + sizeof(uint64_t) * kMaxStages + sizeof(float) * C::RED_FLOATS;
+  const size_t score = sizeof(float) * (size_t)score_scratch_floats(p, D);
+  const size_t smem = ring > score ? ring : score;
   auto kern = pool_score_topk_kernel<T, D, BLK>;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  dim3 grid(p.n_q, p.BH);
-  kern<<<grid, kThreads, smem, s>>>(static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-                                    p, w);
-  return cudaGetLastError();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  int grid = device_sm_count() * per_sm;
+  // the grid barrier needs every CTA resident at once: cooperative launch guarantees it
+  Plan pp = p;
+  Work ww = w;
+  const T* qq = static_cast<const T*>(q);
+  const T* kk = static_cast<const T*>(k);
+  const T* vv = static_cast<const T*>(v);
+  void* args[] = {&qq, &kk, &vv, &pp, &ww};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kern), dim3(grid), dim3(kThreads), args, smem, s);
 }
 
 }  // namespace
+
+size_t pool_partial_floats(const Plan& p) {
+  return (size_t)p.BH * ((p.n_src + kRows - 1) / kRows) * p.n_ctx;
+}
 
 cudaError_t launch_pool_score_topk(const void* q, const void* k, const void* v, const Plan& p, const Work& w,
                                    cudaStream_t s) {
@@ -241,8 +316,7 @@ cudaError_t launch_pool_score_topk(const void* q, const void* k, const void* v, 
     return p.b == 128 ? launch_t<__nv_bfloat16, 64, 128>(q, k, v, p, w, s)
                       : launch_t<__nv_bfloat16, 64, 64>(q, k, v, p, w, s);
   }
-  if (p.D == 128) return p.b == 128 ? launch_t<float, 128, 128>(q, k, v, p, w, s)
-                                    : launch_t<float, 128, 64>(q, k, v, p, w, s);
+  if (p.D != 64) return cudaErrorNotSupported;  // float32 inputs are supported with D = 64 only
   return p.b == 128 ? launch_t<float, 64, 128>(q, k, v, p, w, s) : launch_t<float, 64, 64>(q, k, v, p, w, s);
 }
 

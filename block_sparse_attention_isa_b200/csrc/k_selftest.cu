@@ -2,6 +2,7 @@
 // satisfied must give up on its own, record the failure in the error word and
 // return, leaving the CUDA context usable. This is how every wait in the
 // library behaves when a logic error would otherwise leave it spinning.
+#include "exp2_poly.cuh"
 #include "isa_internal.h"
 #include "ptx.cuh"
 
@@ -17,7 +18,21 @@ __global__ void wait_selftest_kernel(uint32_t* err, uint64_t timeout_ns) {
   if (!mbar_wait(&bar, 0, timeout_ns)) atomicOr(err, kErrSelftest);
 }
 
+// The polynomial 2^x used by the attention softmax, next to CUDA's exp2f, for testing.
+__global__ void exp2_selftest_kernel(const float* x, float* y_poly, float* y_ref, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  y_poly[i] = exp2_poly(x[i]);
+  y_ref[i] = exp2f(x[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, s>>>(x, y_poly, y_ref, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_wait_selftest(uint32_t* err, int timeout_ms, cudaStream_t s) {
   wait_selftest_kernel<<<1, 32, 0, s>>>(err, (uint64_t)timeout_ms * 1000000ull);

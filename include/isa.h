@@ -154,6 +154,14 @@ ISA_API int isa_debug_pooled(int B, int H, int L_src, int L_ctx, int D, int b, f
 ISA_API int isa_selftest_wait_timeout(void* workspace, int timeout_ms, void* stream);
 
 /*
+ * isa_selftest_exp2 - for testing: y_poly[i] = the polynomial 2^x[i] that the
+ * attention softmax computes on the FMA pipe for part of its exponentials
+ * (round-to-nearest range reduction plus a cubic fitted to 2^f on [-1/2, 1/2]),
+ * y_ref[i] = CUDA's exp2f(x[i]). Device pointers, n floats, enqueued on stream.
+ */
+ISA_API int isa_selftest_exp2(const float* x, float* y_poly, float* y_ref, int n, void* stream);
+
+/*
  * isa_set_stage_events - for live per-kernel timing: while set, every forward
  * call made on this host thread records the 5 given CUDA events (cudaEvent_t
  * handles owned by the caller) on its stream: before the pooling kernel and
@@ -172,9 +180,9 @@ ISA_API int isa_set_stage_events(void* const* events, int n_events);
  *   q, k, v    device inputs [B, H, N, D] (as for isa_forward_ex)
  *   sel        device int32 [B, H, k] output: kept context blocks, ascending
  *   colscore   device float32 [B, H, N_ctx / b] output: context-block scores
- * Scratch (the block means of Q, K, V and per-head counters,
- * 3 * B*H * (N/b) * D * 4 bytes plus 4 bytes per head, each part rounded up
- * to 256 bytes) lives in a fixed 32 MiB device array inside the library, which
+ * Scratch (the block means of Q, K, V, 3 * B*H * (N/b) * D * 4 bytes, plus
+ * small partial sums, counters and control words, each part rounded up to 256
+ * bytes) lives in a fixed 32 MiB device array inside the library, which
  * every GPU that loads the library holds until the process exits. Larger sizes
  * return ISA_ERR_UNSUPPORTED before any GPU work. The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress); make that first

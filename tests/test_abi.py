@@ -32,7 +32,7 @@ def L():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(isa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(isa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_and_binding_agree():
@@ -41,7 +41,7 @@ def test_header_and_binding_agree():
 
 def test_library_exports_every_declared_symbol(L):
     out = subprocess.run(["nm", "-D", "--defined-only", isa.lib_path()], capture_output=True, text=True).stdout
-    exported = set(re.findall(r"\bT (isa_[a-z_]+)\b", out))
+    exported = set(re.findall(r"\bT (isa_[a-z0-9_]+)\b", out))
     for name in declared_functions():
         assert name in exported, name
         assert getattr(L, name) is not None

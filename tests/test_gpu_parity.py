@@ -141,3 +141,19 @@ def test_workspace_errors_on_device():
     with pytest.raises(isa.IsaError) as e:
         isa.forward_into(x, x, x, x, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
     assert e.value.code == -1
+
+
+def test_polynomial_exp2_against_cuda_exp2f():
+    """The softmax's FMA-pipe 2^x stays within 1e-4 relative error of CUDA's exp2f."""
+    import torch
+    import block_sparse_attention_isa_b200 as isa
+    xs = np.concatenate([np.linspace(-124.0, 9.0, 200001), np.random.default_rng(0).uniform(-30, 9, 100000)])
+    x = torch.tensor(xs, dtype=torch.float32, device="cuda")
+    yp, yr = torch.empty_like(x), torch.empty_like(x)
+    assert isa.lib().isa_selftest_exp2(x.data_ptr(), yp.data_ptr(), yr.data_ptr(), x.numel(),
+                                       torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    rel = ((yp.double() - yr.double()).abs() / yr.double()).max().item()
+    assert rel <= 1e-4, rel
+    exact = torch.from_numpy(np.exp2(x.cpu().double().numpy()))
+    assert ((yp.cpu().double() - exact).abs() / exact).max().item() <= 1e-4
