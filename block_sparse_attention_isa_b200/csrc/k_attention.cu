@@ -17,14 +17,13 @@
 //    block takes exactly one path, so there is nothing to merge).
 //
 // Design for sm_100a (prior art on the pages is Triton / TileLang on Hopper):
-//  * one CTA per SM (persistent), 20 warps: warp 0 issues TMA loads, warp 1
+//  * one CTA per SM (persistent), 12 warps: warp 0 issues TMA loads, warp 1
 //    owns TMEM and issues tcgen05.mma from one thread (warps 2-3 idle), warps
-//    4-19 are four softmax warpgroups, two per 128-row query tile: a query row
-//    is shared by two threads, each holding 64 of its 128 scores in registers
-//    (setmaxnreg moves registers from warpgroup 0 to them). The two halves
-//    exchange their partial row maxima through shared memory once per K/V
-//    tile, keep separate partial row sums (added once at the end), and each
-//    rescales and writes its own half of the output columns;
+//    4-7 and 8-11 are two softmax warpgroups, one per 128-row query tile; each
+//    softmax thread owns one query row and keeps its 128 scores in registers
+//    (setmaxnreg moves registers from warpgroup 0 to them);
+//  * P is written and released in two halves (keys 0-63, then 64-127), and the
+//    P V MMAs of a half start as soon as it is released;
 //  * a work item is up to two 128-row query tiles of one head (four blocks
 //    when b = 64), both walking the same K/V tiles, so every K/V tile is
 //    loaded once for 256 query rows;
@@ -47,29 +46,28 @@
 namespace isa {
 namespace {
 
-// Threads per query row in the softmax (1: a thread holds all 128 scores of its
-// row; 2: two threads hold 64 each and exchange partial row maxima). One thread
-// per row measured faster (4.78 ms against 6.05 ms at the 32K-token workload).
-#ifndef ISA_ROW_SPLIT
-#define ISA_ROW_SPLIT 1
-#endif
-constexpr int kSplit = ISA_ROW_SPLIT;
-static_assert(kSplit == 1 || kSplit == 2, "one or two threads per row");
-constexpr int kThreads = 128 + 256 * kSplit;  // warpgroup 0 + kSplit softmax warpgroups per query tile
-// Register budget: the kernel is compiled for kLaunchRegs registers a thread at
-// launch (kThreads x kLaunchRegs <= 65536). Warpgroup 0 (TMA + MMA warps) gives
-// registers back and the softmax warpgroups take them; the two shares add up to
-// at most the launch total, so the increase never waits. The launcher checks the
-// compiled count before every launch.
-constexpr int kLaunchRegs = kSplit == 1 ? 168 : 96;
-constexpr int kLowRegs = kSplit == 1 ? 88 : 64;
-constexpr int kHighRegs = kSplit == 1 ? 208 : 104;
-static_assert(128 * kLowRegs + 256 * kSplit * kHighRegs <= kThreads * kLaunchRegs,
-              "register split exceeds the launch budget");
-constexpr int kCols = 128 / kSplit;  // scores per softmax thread
+// One softmax thread per query row holds all 128 scores of its row. (Two threads
+// per row, exchanging partial maxima through shared memory, measured slower:
+// 6.05 ms against 4.78 ms for the attention kernel at the 32K-token workload.)
+constexpr int kThreads = 384;  // warpgroup 0 (TMA, MMA) + one softmax warpgroup per query tile
+// Register budget: the kernel is compiled for 168 registers a thread at launch
+// (384 x 168 = 64512 of the SM's 65536). Warpgroup 0 (TMA + MMA warps) gives
+// registers back and the two softmax warpgroups take them:
+// 128 x 88 + 256 x 208 = 64512, the same total, so the increase never waits.
+// The launcher checks the compiled count before every launch.
+constexpr int kLaunchRegs = 168;
+constexpr int kLowRegs = 88;
+constexpr int kHighRegs = 208;
+static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
+constexpr int kCols = 128;  // scores per softmax thread
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per K/V tile
-constexpr float kRescaleThreshold = 8.0f;  // log2 domain
+// The running row maximum only moves (and O is rescaled) when a tile's maximum
+// exceeds it by more than this many powers of two; P then stays below 2^this.
+#ifndef ISA_RESCALE_LOG2
+#define ISA_RESCALE_LOG2 8
+#endif
+constexpr float kRescaleThreshold = (float)ISA_RESCALE_LOG2;
 // Share of the exponentials computed by the FMA-pipe polynomial instead of ex2:
 // pair i of a row goes to the polynomial when (i % kPolyDen) < kPolyNum. On B200
 // the softmax is bound by instruction issue, not by the ex2 unit, so the
@@ -102,12 +100,10 @@ struct Bars {
   uint64_t q_full[2];
   uint64_t q_empty;
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], p_ready[2], o_done[2];
+  uint64_t s_full[2], p_half[2][2], o_done[2];  // p_half[t][k]: P of keys 64k..64k+63 written
   uint64_t drain;
-  uint64_t xbar[2];          // per query tile: both column halves (256 threads) have written their partial
   uint32_t tmem_base;
   int abort_flag;
-  float xpart[2][2][2][128];  // [exchange parity][query tile][column half][row]: partial row max or row sum
 };
 
 template <typename T, int D>
@@ -239,7 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->q_full[t], 1);
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_ready[t], 128 * kSplit);
+      mbar_init(&bars->p_half[t][0], 128);
+      mbar_init(&bars->p_half[t][1], 128);
       mbar_init(&bars->o_done[t], 1);
     }
     mbar_init(&bars->q_empty, 1);
@@ -250,8 +247,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->v_empty[s], 1);
     }
     mbar_init(&bars->drain, 1);
-    mbar_init(&bars->xbar[0], 128 * kSplit);
-    mbar_init(&bars->xbar[1], 128 * kSplit);
     bars->abort_flag = 0;
     mbar_fence_init();
   }
@@ -390,9 +385,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_ss_lo<C::kTf32>(d, qa + off, ka + off, HI, C::IDESC_QK, s > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](uint32_t d, uint32_t pa, uint32_t va, uint32_t acc) {
+      // P V over keys [64 half, 64 half + 64) of the tile
+      auto issue_pv = [&](uint32_t d, uint32_t pa, uint32_t va, uint32_t acc, int half) {
 #pragma unroll
-        for (int s = 0; s < C::KS_PV; ++s) {
+        for (int s = half * C::KS_PV / 2; s < (half + 1) * C::KS_PV / 2; ++s) {
           const uint32_t off = C::kVT ? (uint32_t)(((s / 4) * C::VT_CH_STRIDE + (s % 4) * 32) >> 4)
                                       : (uint32_t)((s * C::PV_K * 128) >> 4);
           umma_ts_lo<C::kTf32>(d, pa + s * 8, va + off, HI, C::IDESC_PV, (acc | (uint32_t)s) != 0 ? 1u : 0u);
@@ -435,9 +431,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t va = st ? v_lo1 : v_lo0;
           const uint32_t ka1 = st1 ? k_lo1 : k_lo0;
           const uint32_t acc = j > 0 ? 1u : 0u;
-          // tile 0: P0 V_j, then S0 of the next K/V tile
-          if (!wait_or_abort(&bars->p_ready[0], pv_cnt0 & 1)) break;
-          issue_pv(t_o0, t_s0, va, acc);
+          // tile 0: P0 V_j in two halves (each as soon as its P is written), then S0 of the next K/V tile
+          if (!wait_or_abort(&bars->p_half[0][0], pv_cnt0 & 1)) break;
+          issue_pv(t_o0, t_s0, va, acc, 0);
+          if (!wait_or_abort(&bars->p_half[0][1], pv_cnt0 & 1)) break;
+          issue_pv(t_o0, t_s0, va, 1u, 1);
           umma_commit(&bars->o_done[0]);
           ++pv_cnt0;
           if (more) {
@@ -447,8 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // tile 1
           if (two) {
-            if (!wait_or_abort(&bars->p_ready[1], pv_cnt1 & 1)) break;
-            issue_pv(t_o1, t_s1, va, acc);
+            if (!wait_or_abort(&bars->p_half[1][0], pv_cnt1 & 1)) break;
+            issue_pv(t_o1, t_s1, va, acc, 0);
+            if (!wait_or_abort(&bars->p_half[1][1], pv_cnt1 & 1)) break;
+            issue_pv(t_o1, t_s1, va, 1u, 1);
             umma_commit(&bars->o_done[1]);
             ++pv_cnt1;
             if (more) {
@@ -472,31 +472,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax + epilogue
     regs_alloc<kHighRegs>();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
-    const int sw = warp - 4;
-    const int t = sw / (4 * kSplit);         // query tile
-    const int h = (sw >> 2) % kSplit;        // column part of the scores and of the output
+    const int t = (warp - 4) >> 2;           // query tile of this warpgroup
     const int wl = warp & 3;                 // TMEM lane quarter
     const int row = wl * 32 + lane;          // row inside the 128-row tile
     const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
-    const uint32_t t_s = tmem + lane_off + t * 128 + h * kCols;                               // this thread's scores
-    const uint32_t t_p = tmem + lane_off + t * 128 + h * (sizeof(T) == 2 ? kCols / 2 : kCols);  // its P
-    const uint32_t t_o = tmem + lane_off + 256 + t * 128 + h * (D / kSplit);                  // its O columns
-    uint32_t s_cnt = 0, pv_cnt = 0, x_cnt = 0;
+    const uint32_t t_s = tmem + lane_off + t * 128;        // this row's scores, then its P
+    const uint32_t t_p = t_s;
+    const uint32_t t_o = tmem + lane_off + 256 + t * 128;  // this row's O
+    uint32_t s_cnt = 0, pv_cnt = 0;
     bool ok = true;
     T* out = static_cast<T*>(p.out);
-    // Partial-value exchange with the thread that holds the other half of the row:
-    // write, arrive on the tile's barrier (256 arrivals), wait (bounded), read the
-    // partner's value. Buffers alternate with the exchange count, so a value is only
-    // overwritten after the partner has passed the next exchange.
-    auto exchange = [&](float v, float& partner) -> bool {
-      const uint32_t par = x_cnt & 1;
-      bars->xpart[par][t][h][row] = v;
-      mbar_arrive(&bars->xbar[t]);
-      if (!warp_wait(bars, &bars->xbar[t], par, p.err)) return false;
-      partner = bars->xpart[par][t][h ^ 1][row];
-      ++x_cnt;
-      return true;
-    };
     for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x) {
       const Item it = decode_item(p, g);
       if (t >= it.ntiles) continue;
@@ -511,61 +496,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j == it.nkv - 1 && it.last_valid < kBN) {  // ragged last K/V tile (uniform branch)
 #pragma unroll
           for (int i = 0; i < kCols; ++i)
-            if (h * kCols + i >= it.last_valid) r[i] = __float_as_uint(-INFINITY);
+            if (i >= it.last_valid) r[i] = __float_as_uint(-INFINITY);
         }
-        // (partial) row max of the raw scores: 4 independent chains of 3-input max
-        float mc[4];
+        // row max of the raw scores: 8 independent chains of 3-input max
+        float mc[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) mc[c] = __uint_as_float(r[c]);
+        for (int c = 0; c < 8; ++c) mc[c] = __uint_as_float(r[c]);
 #pragma unroll
-        for (int i = 4; i < kCols; i += 8) {
+        for (int i = 8; i < kCols; i += 16) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[i + c]), __uint_as_float(r[i + 4 + c]));
+          for (int c = 0; c < 8; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[i + c]), __uint_as_float(r[i + 8 + c]));
         }
-        float pm = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
-        if constexpr (kSplit == 2) {
-          // exchange with the thread holding the other half of the row (the exchange also
-          // guarantees that both halves have read their scores before P overwrites them)
-          float pm_other;
-          if (!exchange(pm, pm_other)) { ok = false; break; }
-          pm = fmaxf(pm, pm_other);
-        }
-        const float mx = pm * p.scale_log2;
+        const float mx = fmaxf(fmax3(mc[0], mc[1], mc[2]), fmax3(fmax3(mc[3], mc[4], mc[5]), mc[6], mc[7])) *
+                         p.scale_log2;
         // lazy max: move it only when the tile's max exceeds it by more than 2^8
         const bool need = (j > 0) && (mx > m + kRescaleThreshold);
         const float alpha = need ? ex2_approx(m - mx) : 1.0f;
         if (j == 0 || need) m = mx;
-        // p = 2^(s * scale - m), in pairs; one pair in kPolyEvery on the FMA pipe, the rest on ex2
-        const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(-m, -m);
-        uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int i = 0; i < kCols / 2; ++i) {
-          const uint64_t x = ffma2(static_cast<uint64_t>(r[2 * i]) | (static_cast<uint64_t>(r[2 * i + 1]) << 32), sc2,
-                                   nm2);
-          uint64_t e;
-          if (i % kPolyDen < kPolyNum) e = exp2_poly2(x);
-          else e = pack2(ex2_approx(lo2(x)), ex2_approx(hi2(x)));
-          acc[i & 3] = fadd2(acc[i & 3], e);
-          if constexpr (sizeof(T) == 2) {
-            __nv_bfloat162 hv = __floats2bfloat162_rn(lo2(e), hi2(e));
-            r[i] = *reinterpret_cast<uint32_t*>(&hv);
-          } else {
-            r[2 * i] = static_cast<uint32_t>(e);
-            r[2 * i + 1] = static_cast<uint32_t>(e >> 32);
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < (sizeof(T) == 2 ? kCols / 64 : kCols / 32); ++c) tmem_st32(t_p + 32 * c, r + 32 * c);
-        const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-        l = l * alpha + (lo2(a2) + hi2(a2));
-        // O holds P V up to tile j-1; rows whose max moved are rescaled in place
-        // (this half's columns) before P V of tile j may start. TMEM moves are
-        // warp-collective, so the whole warp takes this step when any of its rows
-        // needs it (alpha = 1 for the others).
+        // O holds P V up to tile j-1 (complete: this tile's S was committed after it);
+        // rows whose max moved are rescaled in place before any P of tile j is
+        // released. TMEM moves are warp-collective, so the whole warp takes this step
+        // when any of its rows needs it (alpha = 1 for the others).
         if (__any_sync(0xffffffffu, need)) {
           if (!warp_wait(bars, &bars->o_done[t], (pv_cnt - 1) & 1, p.err)) { ok = false; break; }
 #pragma unroll 1
-          for (int c = 0; c < D / 32 / kSplit; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
             tmem_ld32(t_o + 32 * c, o);
             tmem_ld_wait<32>(o);
@@ -574,26 +529,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(t_o + 32 * c, o);
           }
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bars->p_ready[t]);
+        // p = 2^(s * scale - m), in pairs (pairs with i % kPolyDen < kPolyNum on the FMA
+        // pipe, the rest on ex2). P is written and released in two halves (keys 0-63,
+        // then 64-127) so that the P V MMAs can start on the first half.
+        const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(-m, -m);
+        uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int i = half * kCols / 4; i < (half + 1) * kCols / 4; ++i) {
+            const uint64_t x = ffma2(static_cast<uint64_t>(r[2 * i]) | (static_cast<uint64_t>(r[2 * i + 1]) << 32), sc2,
+                                     nm2);
+            uint64_t e;
+            if (i % kPolyDen < kPolyNum) e = exp2_poly2(x);
+            else e = pack2(ex2_approx(lo2(x)), ex2_approx(hi2(x)));
+            acc[i & 3] = fadd2(acc[i & 3], e);
+            if constexpr (sizeof(T) == 2) {
+              __nv_bfloat162 hv = __floats2bfloat162_rn(lo2(e), hi2(e));
+              r[i] = *reinterpret_cast<uint32_t*>(&hv);
+            } else {
+              r[2 * i] = static_cast<uint32_t>(e);
+              r[2 * i + 1] = static_cast<uint32_t>(e >> 32);
+            }
+          }
+          // this half's P: bf16 pairs in kCols/4 columns, or fp32 in kCols/2 columns
+          constexpr int kPCols = sizeof(T) == 2 ? kCols / 4 : kCols / 2;
+#pragma unroll
+          for (int c = 0; c < kPCols / 32; ++c) {
+            const int col = half * kPCols + 32 * c;
+            tmem_st32(t_p + col, r + col);
+          }
+          static_assert(kPCols % 32 == 0, "P columns");
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&bars->p_half[t][half]);
+        }
+        const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+        l = l * alpha + (lo2(a2) + hi2(a2));
         ++pv_cnt;
       }
       if (!ok) break;
       // epilogue: O / (l_half0 + l_half1) for this half's columns, at the row's original token position
-      if constexpr (kSplit == 2) {
-        float l_other;
-        if (!exchange(l, l_other)) { ok = false; break; }
-        l += l_other;
-      }
       const float inv_l = 1.0f / l;
       if (!warp_wait(bars, &bars->o_done[t], (pv_cnt - 1) & 1, p.err)) { ok = false; break; }
       const int u = t * p.bpt + row / p.b;
       const bool store = (u < it.nblk);
       const size_t token = (size_t)it.blk(store ? u : 0) * p.b + (row % p.b);
-      T* dst = out + ((size_t)it.bh * p.N + token) * D + h * (D / kSplit);
+      T* dst = out + ((size_t)it.bh * p.N + token) * D;
 #pragma unroll 1
-      for (int c = 0; c < D / 32 / kSplit; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(t_o + 32 * c, o);
         tmem_ld_wait<32>(o);

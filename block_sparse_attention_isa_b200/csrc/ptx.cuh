@@ -271,11 +271,6 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Named barrier `id` (1..15) over `count` threads (a multiple of 32, whole warps).
-__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // Per-warpgroup register budget changes (all 128 threads of the warpgroup execute them).
 template <uint32_t kRegs>
 __device__ __forceinline__ void regs_dealloc() {
