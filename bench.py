@@ -143,8 +143,11 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- arms
 
-def workload_inputs(w, seed=0):
-    att = isa_synth.attempts_for(w, seed)
+def workload_inputs(w, seed=0, full=None):
+    """Q, K, V of workload w; with `full` (w = full with fewer heads) its first heads, same draws."""
+    att = isa_synth.attempts_for(full or w, seed)
+    if att is not None and full is not None:
+        att = att[:, :w.H]
     return isa_synth.make_inputs(w, seed, att)
 
 
@@ -168,30 +171,52 @@ def cpu_oracle_sample(w, q, k, v, heads, seconds_cap=60.0):
 
 
 def run_reference(args, w):
-    """The CPU oracle as it stands, one head of the workload per step."""
+    """The CPU oracle as it stands. Each step is a bounded sample of the workload: the context
+    selection and routing of one head, then the output rows of every eighth query block of that
+    head (both paths in their natural proportion); the work counted is exactly that sample's."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    q, k, v = isa_synth.make_inputs(w, 0, isa_synth.attempts_for(w, 0), heads=[(0, h) for h in range(w.H)][:max(1, args.steps + args.warmup)])
+    import numpy as np
     from oracle import isa_oracle as O
-    f_head = flops_per_call(w)["total"] / (w.B * w.H)
+    n_heads = min(w.B * w.H, max(1, args.steps + args.warmup))
+    att = isa_synth.attempts_for(getattr(args, "full_workload", None) or w, 0)
+    if att is not None:
+        att = att[:, :w.H]
+    q, k, v = isa_synth.make_inputs(w, 0, att, heads=[(0, h) for h in range(n_heads)])
+    parts = 8
+    n_q = w.N // w.b
+    kk = O.kept_context_blocks(w.alpha_s, w.L_ctx // w.b)
+    n_new = w.L_src // w.b + kk
+    per_head = O.executed_flops(1, 1, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, w.alpha_f)
+    sel_route_flops = per_head["coarse"] + per_head["route"]
+
+    def step(s):
+        h = s % n_heads
+        sr = O.isa_select_route_ref(q[0, h], k[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+        blocks = np.arange(s % parts, n_q, parts)
+        rows = (blocks[:, None] * w.b + np.arange(w.b)[None, :]).ravel()
+        O.isa_rows_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, rows, sr=sr)
+        taylor = set(int(t) for t in sr["taylor"])
+        n_t = sum(int(bl) in taylor for bl in blocks)
+        return sel_route_flops + 4.0 * w.b * w.D * ((len(blocks) - n_t) * n_new * w.b + n_t * n_new)
+
     for s in range(args.warmup):
-        O.isa_slice_ref(q[0, s % w.H], k[0, s % w.H], v[0, s % w.H], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+        step(s)
     t0 = time.perf_counter()
-    for s in range(args.steps):
-        h = (args.warmup + s) % w.H
-        O.isa_slice_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+    flops = sum(step(args.warmup + s) for s in range(args.steps))
     dt = time.perf_counter() - t0
-    value = f_head * args.steps / dt / 1e12
+    value = flops / dt / 1e12
     cores = os.cpu_count()
+    sample = (f"per step: selection and routing of one head, then the rows of every {parts}th query block "
+              f"of it ({args.steps} steps over {n_heads} of {w.B * w.H} heads)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "b": w.b,
-                       "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "sample": "one head per step"},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{args.steps} heads of {w.B * w.H}, one per step"},
+            "config": {"workload": w.name + (f" (first {w.H} heads)" if args.heads else ""), "B": w.B, "H": w.H,
+                       "N": w.N, "D": w.D, "b": w.b, "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -214,7 +239,7 @@ def run_ours(args, w):
     dev = torch.device("cuda", local)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
-    q, k, v = workload_inputs(w)
+    q, k, v = workload_inputs(w, full=getattr(args, "full_workload", None))
     tq, tk, tv = (torch.from_numpy(x).to(dev, dt) for x in (q, k, v))
     out = torch.empty_like(tq)
     ws = torch.empty(isa.workspace_bytes(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s,
@@ -274,7 +299,7 @@ def run_ours(args, w):
 
     # end to end through the host-buffer entry point (pinned host memory, copies inside the timed region)
     e2e = None
-    if rank == 0 or world > 1:
+    if not args.no_e2e and (rank == 0 or world > 1):
         hq, hk, hv = (t.cpu().pin_memory() for t in (tq, tk, tv))
         hout = torch.empty_like(hq).pin_memory()
         n_e2e = max(1, min(args.steps, 5))
@@ -303,7 +328,7 @@ def run_ours(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
             "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "b": w.b,
+            "config": {"workload": w.name + (f" (first {w.H} heads)" if args.heads else ""), "B": w.B, "H": w.H, "N": w.N, "D": w.D, "b": w.b,
                        "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "global_batch": w.B * world,
                        "seq_len": w.N, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (Q, K, V = %.2f GB per step)" % (3 * tq.numel() * tq.element_size() / 1e9)},
@@ -330,14 +355,21 @@ def run_ours(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=isa_synth.HEADLINE)
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only the first H heads of the workload (small profiling captures; not a bench line)")
     args = ap.parse_args()
     w = isa_synth.all_workloads()[args.workload]
+    args.full_workload = None
+    if args.heads:
+        args.full_workload = w
+        w = w.with_(H=min(args.heads, w.H))
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args, w)
