@@ -183,7 +183,9 @@ int run_forward(const void* q, const void* k, const void* v, const Plan& p, void
   if ((e = launch_route(p, w, s)) != cudaSuccess) return cuda_fail(e, "routing launch");
   if ((e = launch_transpose_v(v, p, w, s)) != cudaSuccess) return cuda_fail(e, "V transpose launch");
   if ((e = mark(3, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
-  if ((e = launch_attention(q, k, v, out, p, w, s, nullptr)) != cudaSuccess) return cuda_fail(e, "attention launch");
+  e = attention_pair_supported(p) ? launch_attention_pair(q, k, v, out, p, w, s, nullptr)
+                                  : launch_attention(q, k, v, out, p, w, s, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   if ((e = mark(4, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
   if (dbg_sel && p.k > 0) {
     e = cudaMemcpyAsync(dbg_sel, w.sel, sizeof(int32_t) * (size_t)p.BH * p.k, cudaMemcpyDeviceToDevice, s);

@@ -82,6 +82,10 @@ cudaError_t launch_route(const Plan& p, const Work& w, cudaStream_t s);
 cudaError_t launch_transpose_v(const void* v, const Plan& p, const Work& w, cudaStream_t s);
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out, const Plan& p,
                              const Work& w, cudaStream_t s, int* n_ctas_out);
+// Attention on pairs of CTAs (bf16, D = 128): same contract as launch_attention.
+bool attention_pair_supported(const Plan& p);
+cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, void* out, const Plan& p,
+                                  const Work& w, cudaStream_t s, int* n_ctas);
 
 // One thread waits on an mbarrier that nothing arrives on; the bounded wait gives
 // up after `timeout_ms` and sets kErrSelftest in err[0].

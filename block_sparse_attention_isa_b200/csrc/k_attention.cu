@@ -42,6 +42,7 @@
 #include "exp2_poly.cuh"
 #include "isa_internal.h"
 #include "ptx.cuh"
+#include "tensor_map.cuh"
 
 namespace isa {
 namespace {
@@ -187,7 +188,7 @@ __device__ __forceinline__ void raise_abort(Bars* b, uint32_t* err, uint32_t cod
 // All 32 lanes wait on the barrier; the result is the same in every lane and the
 // warp is converged on return (the TMEM moves that follow are warp-collective).
 __device__ __forceinline__ bool warp_wait(Bars* b, uint64_t* bar, uint32_t parity, uint32_t* err) {
-  bool ok = !aborted(b) && mbar_wait(bar, parity);
+  bool ok = mbar_wait_or_abort(bar, parity, &b->abort_flag);
   ok = __all_sync(0xffffffffu, ok);
   if (!ok) raise_abort(b, err, kErrSoftmax);
   tc_fence_after();
@@ -395,8 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       auto wait_or_abort = [&](uint64_t* bar, uint32_t par) -> bool {
-        if (aborted(bars)) { ok = false; return false; }
-        if (!mbar_wait(bar, par)) { raise_abort(bars, p.err, kErrMma); ok = false; return false; }
+        if (!mbar_wait_or_abort(bar, par, &bars->abort_flag)) { raise_abort(bars, p.err, kErrMma); ok = false; return false; }
         tc_fence_after();
         return true;
       };
@@ -596,48 +596,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(*reinterpret_cast<volatile uint32_t*>(&bars->tmem_base), 512);
   }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// [heads][rows][D] view, box of 64 rows x one 128-byte chunk, 128-byte swizzle,
-// out-of-range rows read as zeros.
-bool make_map(CUtensorMap* m, const void* base, int elem, int D, int rows, int heads) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const CUtensorMapDataType dt = elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads};
-  cuuint64_t strides[2] = {(cuuint64_t)D * elem, (cuuint64_t)rows * D * elem};
-  cuuint32_t box[3] = {(cuuint32_t)(128 / elem), 64u, 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-// fp32 [heads][D][keys] view of a transposed V, box of 32 keys x D rows, 128-byte swizzle,
-// keys past the end read as zeros.
-bool make_map_t(CUtensorMap* m, const void* base, int keys, int ld, int D, int heads) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)keys, (cuuint64_t)D, (cuuint64_t)heads};
-  cuuint64_t strides[2] = {(cuuint64_t)ld * 4, (cuuint64_t)ld * D * 4};
-  cuuint32_t box[3] = {32u, (cuuint32_t)D, 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
 }
 
 template <typename T, int D>

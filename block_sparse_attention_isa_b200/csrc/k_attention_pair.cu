@@ -1,0 +1,658 @@
+// Stage 4-5 of In-context Sparse Attention (both attention paths and the
+// write-back) for bf16 inputs with D = 128, on pairs of CTAs that share every
+// tensor-core operation.
+//
+// Method: "Lightning Unified Video Editing via In-Context Sparse Attention",
+// papernotes.org notes, Key design 2 and the flowchart: the exact path is online
+// softmax attention of a sharp query block over all keys of
+// K_new = [K_src ; kept context blocks]; the block-wise 0th-order Taylor path
+// replaces each block j of K_new by b * exp(q . Kc_j / sqrt(D)) paired with Vc_j,
+// and since every block holds b keys the weight b cancels, leaving
+// softmax(q Kc_new^T / sqrt(D)) Vc_new: the same attention against the n_new
+// pooled rows. Each output row is written at its original token position.
+//
+// Why pairs. With one CTA per SM, every 256 query rows re-read their head's whole
+// K_new / V_new from L2 (22.5 GB per call at the 32K-token workload) and the
+// Q K^T MMAs read 8 KB of shared memory per 64 cycles, the tensor core's whole
+// shared-memory rate, so the K/V stream and the MMAs slow each other down. A
+// tcgen05.mma with cta_group::2 computes M = 256 rows on two SMs: each CTA holds
+// its own 128 query rows of A and HALF of B. Here each CTA loads 32 of the 64
+// keys of every K tile and 64 of the 128 columns of every V tile, so per query
+// row the pair moves half the K/V bytes from L2 and reads half the B operand
+// bytes from shared memory.
+//
+// Structure (each CTA of the pair: 12 warps, one CTA per SM):
+//  * warp 0 issues the TMA loads of this CTA's halves; the loads of both CTAs
+//    signal the leader CTA's "full" barriers, which the leader arms with the
+//    byte count of both halves;
+//  * warp 1 of the leader issues every MMA from one thread; completions are
+//    committed to the barriers of both CTAs at once (multicast commit);
+//  * warps 4-7 and 8-11 are two softmax warpgroups per CTA, one per query-tile
+//    slot: slot t of a work item is tile 2t in the leader and tile 2t + 1 in the
+//    peer (a slot with no tile for the peer gives it a copy of the leader's tile,
+//    computed and not stored). One thread per query row; every softmax thread of
+//    both CTAs arrives on the leader's "P written" barrier;
+//  * K/V tiles of 64 keys in 8-stage rings; TMEM of each CTA: slot t owns two
+//    64-column S buffers at [128 t, 128 t + 128) and O_t at [256 + 128 t, ...);
+//    S of K/V tile n goes to buffer n % 2, P_n is written over it as bf16 pairs
+//    and read by the P V MMA straight from TMEM;
+//  * MMA order per K/V tile j: P0 V_j, S0 of tile j + 2, P1 V_j, S1 of tile j + 2,
+//    so the softmax of tile j + 1 never waits for the P V of tile j;
+//  * lazy rescaling (the running max moves only when it grows by more than 2^8),
+//    exact items first and Taylor items after in the static schedule;
+//  * every wait is bounded; on a timeout the CTA flags an error in the device
+//    error word and in the abort flags of both CTAs, lets its copies land,
+//    meets its peer at a cluster barrier and frees TMEM.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <float.h>
+
+#include "exp2_poly.cuh"
+#include "isa_internal.h"
+#include "ptx.cuh"
+#include "tensor_map.cuh"
+
+namespace isa {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;
+constexpr int kLowRegs = 88;
+constexpr int kHighRegs = 208;
+static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
+constexpr int kD = 128;
+constexpr int kBM = 128;            // query rows per tile (per CTA)
+constexpr int kBN = 64;             // keys per K/V tile (per pair)
+constexpr int kCols = kBN;          // scores per softmax thread and K/V tile
+constexpr int kStages = 8;   // K/V ring: stage i holds this CTA's halves of the K and V tile i
+constexpr int kRB = kD * 2;         // bytes per row
+constexpr int kQCh = kBM * 128;     // bytes between the two 128-byte chunks of a Q tile
+constexpr int kQTile = kBM * kRB;   // 32 KB
+constexpr int kKRows = kBN / 2;     // keys of each K tile held by one CTA
+constexpr int kKCh = kKRows * 128;  // bytes between the chunks of a K half-tile
+constexpr int kKHalf = kKRows * kRB;  // 8 KB
+constexpr int kVHalf = kBN * 128;     // 8 KB: 64 keys x this CTA's 64 columns
+constexpr uint32_t kIdescQK = umma_idesc(1u, 256, kBN, 0, 0);
+constexpr uint32_t kIdescPV = umma_idesc(1u, 256, kD, 0, 1);
+constexpr float kRescaleThreshold = 8.0f;
+// Share of the exponentials computed by the FMA-pipe polynomial (exp2_poly.cuh) instead of
+// ex2: pair i of a row goes to the polynomial when (i % kPolyDen) < kPolyNum.
+#ifndef ISA_PAIR_POLY_NUM
+#define ISA_PAIR_POLY_NUM 0
+#endif
+#ifndef ISA_PAIR_POLY_DEN
+#define ISA_PAIR_POLY_DEN 8
+#endif
+constexpr int kPolyNum = ISA_PAIR_POLY_NUM;
+constexpr int kPolyDen = ISA_PAIR_POLY_DEN;
+
+struct PairParams {
+  const int32_t* route;
+  void* out;
+  uint32_t* err;
+  int BH, N, b, L_src, n_q, n_exact, n_flat, L_new, n_new;
+  int bpt;      // blocks per 128-row tile (128 / b)
+  int bpi;      // blocks per work item (4 tiles)
+  int items_e;  // exact items per head
+  int items_t;  // Taylor items per head
+  int total;    // all items
+  float scale_log2;
+};
+
+struct Bars {
+  uint64_t q_full[2];    // leader: Q of slot t in both CTAs
+  uint64_t q_empty[2];   // slot t's S MMAs of the item are complete
+  uint64_t kv_full[kStages];   // leader: both CTAs' K and V halves of the stage
+  uint64_t kv_empty[kStages];  // both MMA issuers are done with the stage (2 arrivals)
+  uint64_t s_full[2][2];  // [slot][S buffer]
+  uint64_t p_full[2][2];  // leader: [slot][S buffer], one arrival per softmax thread of both CTAs
+  uint64_t o_done[2][2];  // [slot][S buffer]: the P V MMAs of the K/V tiles in this buffer are complete
+  uint64_t drain[2];      // leader: every MMA of issuer t is complete
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+constexpr int kOffQ = 0;
+constexpr int kOffK = 2 * kQTile;
+constexpr int kOffV = kOffK + kStages * kKHalf;
+constexpr int kOffBar = kOffV + kStages * kVHalf;
+constexpr int kSmemAlloc = kOffBar + (int)sizeof(Bars) + 1024;
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
+
+// ---------------------------------------------------------------- CTA-pair PTX
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_warp() {  // whole warp
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+// Arrive on a barrier of either CTA. Default (release, CTA scope) semantics: what the
+// barrier hands over is TMEM data, ordered by tcgen05.wait::st and the tcgen05 fences
+// around the barrier; a cluster-scope release here measured 1.4x slower for the kernel.
+__device__ __forceinline__ void arrive_cluster(uint32_t addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+__device__ __forceinline__ void store_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// TMA load into this CTA's shared memory, completion counted on a barrier of the leader CTA.
+__device__ __forceinline__ void tma_load_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+// Arrive on `bar` in both CTAs once every MMA issued so far is complete.
+__device__ __forceinline__ void commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_addr(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ss_pair(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc,
+                                            uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .b64 da, db;\n\t.reg .pred p;\n\tmov.b64 da, {%1, %5};\n\tmov.b64 db, {%2, %5};\n\t"
+      "setp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %3, p;\n\t}\n" ::"r"(d),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(acc), "r"(hi)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_pair(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t hi, uint32_t idesc,
+                                            uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .b64 db;\n\t.reg .pred p;\n\tmov.b64 db, {%2, %5};\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], db, %3, p;\n\t}\n" ::"r"(d),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(acc), "r"(hi)
+      : "memory");
+}
+
+struct Item {
+  int bh, kind, nblk, ntiles, nslots, nkv, last_valid;
+  const int32_t* lst;
+  __device__ __forceinline__ int blk(int u) const { return __ldg(lst + u); }
+};
+
+__device__ __forceinline__ Item decode_item(const PairParams& p, int g) {
+  Item it;
+  int count, base, pp;
+  if (g < p.BH * p.items_e) {
+    it.bh = g / p.items_e;
+    pp = g - it.bh * p.items_e;
+    it.kind = 0;
+    count = p.n_exact;
+    base = 0;
+  } else {
+    const int g2 = g - p.BH * p.items_e;
+    it.bh = g2 / p.items_t;
+    pp = g2 - it.bh * p.items_t;
+    it.kind = 1;
+    count = p.n_flat;
+    base = p.n_exact;
+  }
+  const int first = pp * p.bpi;
+  it.lst = p.route + (size_t)it.bh * p.n_q + base + first;
+  it.nblk = min(p.bpi, count - first);
+  it.ntiles = (it.nblk + p.bpt - 1) / p.bpt;
+  it.nslots = (it.ntiles + 1) / 2;
+  const int rows = it.kind == 0 ? p.L_new : p.n_new;
+  it.nkv = (rows + kBN - 1) / kBN;
+  it.last_valid = rows - kBN * (it.nkv - 1);
+  return it;
+}
+
+// Record the error and stop both CTAs of the pair.
+__device__ __noinline__ void raise_abort(Bars* b, uint32_t* err, uint32_t code) {
+  atomicOr(err, code);
+  *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
+  store_cluster_u32(map_to(&b->abort_flag, cluster_rank() ^ 1u), 1u);
+}
+
+// All 32 lanes wait on a local barrier; the warp is converged on return.
+__device__ __forceinline__ bool warp_wait(Bars* b, uint64_t* bar, uint32_t parity, uint32_t* err) {
+  bool ok = mbar_wait_or_abort(bar, parity, &b->abort_flag);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok) raise_abort(b, err, kErrSoftmax);
+  tc_fence_after();
+  return ok;
+}
+
+__device__ __forceinline__ void store_row_chunk(__nv_bfloat16* dst, const float* v) {  // 32 values
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    pk[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    attention_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_ksel, const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_vsel, const __grid_constant__ CUtensorMap tm_kcn,
+                          const __grid_constant__ CUtensorMap tm_vcn, const PairParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + kOffQ;
+  uint8_t* sK = smem + kOffK;
+  uint8_t* sV = smem + kOffV;
+  Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->q_full[t], 1);
+      mbar_init(&bars->q_empty[t], 1);
+      mbar_init(&bars->drain[t], 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&bars->s_full[t][b], 1);
+        mbar_init(&bars->p_full[t][b], 256);
+        mbar_init(&bars->o_done[t][b], 1);
+      }
+    }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 2);
+    }
+    bars->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_ksel);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_vsel);
+    tma_prefetch_desc(&tm_kcn);
+    tma_prefetch_desc(&tm_vcn);
+  }
+  if (warp == 1) {  // the same warp in both CTAs allocates the pair's TMEM
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(&bars->tmem_base)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_warp();  // barriers initialised and TMEM allocated in both CTAs
+  tc_fence_after();
+
+  if (warp < 4) regs_dealloc<kLowRegs>();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      const uint32_t q_full_l = map_to(&bars->q_full[0], 0);
+      const uint32_t kv_full_l = map_to(&bars->kv_full[0], 0);
+      uint32_t kv_it = 0, q_loads0 = 0, q_loads1 = 0;
+      bool ok = true;
+      for (int g = pair; g < p.total && ok; g += npairs) {
+        const Item it = decode_item(p, g);
+        for (int t = 0; t < it.nslots; ++t) {
+          // slot t's Q buffer is free once the S MMAs of the last item that used it are complete
+          const uint32_t prior = t == 0 ? q_loads0 : q_loads1;
+          if (prior > 0 && !mbar_wait(&bars->q_empty[t], (prior - 1) & 1)) {
+            raise_abort(bars, p.err, kErrProducer);
+            ok = false;
+            break;
+          }
+          if (t == 0) ++q_loads0; else ++q_loads1;
+          if (rank == 0) mbar_arrive_expect_tx(&bars->q_full[t], 2 * kQTile);
+          int ut = 2 * t + (int)rank;
+          if (ut >= it.ntiles) ut = 2 * t;  // no tile for the peer in this slot: a copy, not stored
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int r = 64 * h;
+            int u = ut * p.bpt + r / p.b;
+            if (u >= it.nblk) u = ut * p.bpt;  // missing block of a partial tile: rows are not stored
+            const int y = it.blk(u) * p.b + (r % p.b);
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              tma_load_pair(sQ + t * kQTile + c * kQCh + h * 8192, &tm_q, q_full_l + 8u * t, c * 64, y, it.bh);
+          }
+        }
+        for (int j = 0; j < it.nkv && ok; ++j, ++kv_it) {
+          if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) { ok = false; break; }
+          const int r0 = j * kBN;
+          const int st = kv_it % kStages;
+          if (!mbar_wait(&bars->kv_empty[st], ((kv_it / kStages) & 1) ^ 1)) {
+            raise_abort(bars, p.err, kErrProducer);
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&bars->kv_full[st], 2 * (kKHalf + kVHalf));
+          const uint32_t bar = kv_full_l + 8u * st;
+          // K: this CTA's 32 keys of the tile (a 64-key tile never straddles the source/context seam)
+          {
+            const int rk = r0 + (int)rank * kKRows;
+            const CUtensorMap* map;
+            int y;
+            if (it.kind == 0) {
+              if (rk < p.L_src) { map = &tm_k; y = rk; } else { map = &tm_ksel; y = rk - p.L_src; }
+            } else {
+              map = &tm_kcn; y = rk;
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c) tma_load_pair(sK + st * kKHalf + c * kKCh, map, bar, c * 64, y, it.bh);
+          }
+          // V: all 64 keys, this CTA's 64 columns
+          {
+            const CUtensorMap* map;
+            int y;
+            if (it.kind == 0) {
+              if (r0 < p.L_src) { map = &tm_v; y = r0; } else { map = &tm_vsel; y = r0 - p.L_src; }
+            } else {
+              map = &tm_vcn; y = r0;
+            }
+            tma_load_pair(sV + st * kVHalf, map, bar, (int)rank * 64, y, it.bh);
+          }
+        }
+      }
+      if (!ok) {
+        // the copies this thread started signal the leader's barriers, which this CTA cannot
+        // wait on; give them time to land (copies complete in microseconds) before leaving
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 2000000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers (leader CTA only)
+    // Warp 1 issues the MMAs of slot 0 and warp 2 those of slot 1. The two streams are
+    // independent, so while one thread waits for a barrier the other keeps the tensor
+    // core busy (the issuing thread stalls on its barrier reads, and the MMA pipe holds
+    // little queued work). Both release each K/V stage (2 arrivals), so a thread whose
+    // slot is empty in an item still walks the item's stages, waiting for each to fill
+    // before releasing it: it can never release a stage ahead of the other thread.
+    if (rank == 0 && lane == 0) {
+      const int t = warp - 1;
+      const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
+      uint32_t kv_base = 0, q_cnt = 0, s_seq = 0, p_seq = 0;
+      bool ok = true;
+      constexpr uint32_t HI = desc_hi_sw128(1024);
+      const uint32_t q_lo = desc_lo(smem_addr(sQ + t * kQTile), 16);
+      const uint32_t k_lo = desc_lo(smem_addr(sK), 16);
+      const uint32_t v_lo = desc_lo(smem_addr(sV), (uint32_t)kVHalf);
+      const uint32_t t_s = tmem + 128 * t, t_o = tmem + 256 + 128 * t;
+      // S = Q_t K^T for the K tile in stage st (rows of both CTAs, keys of both halves), into S buffer s_seq & 1
+      auto issue_s = [&](uint32_t st) {
+        const uint32_t d = t_s + (s_seq & 1) * kBN;
+        const uint32_t kb = k_lo + ((st * kKHalf) >> 4);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const uint32_t qo = (uint32_t)(((s / 4) * kQCh + (s % 4) * 32) >> 4);
+          const uint32_t ko = (uint32_t)(((s / 4) * kKCh + (s % 4) * 32) >> 4);
+          mma_ss_pair(d, q_lo + qo, kb + ko, HI, kIdescQK, s > 0 ? 1u : 0u);
+        }
+        commit_pair(&bars->s_full[t][s_seq & 1]);
+        ++s_seq;
+      };
+      // O_t (+)= P V for the V tile in stage st, P (of each CTA, from its own TMEM) in S buffer p_seq & 1
+      auto issue_pv = [&](uint32_t st, uint32_t acc) {
+        const uint32_t pa = t_s + (p_seq & 1) * kBN;
+        const uint32_t vb = v_lo + ((st * kVHalf) >> 4);
+#pragma unroll
+        for (int s = 0; s < kBN / 16; ++s)
+          mma_ts_pair(t_o, pa + s * 8, vb + (uint32_t)((s * 16 * 128) >> 4), HI, kIdescPV,
+                      (acc | (uint32_t)s) != 0 ? 1u : 0u);
+        commit_pair(&bars->o_done[t][p_seq & 1]);
+        ++p_seq;
+      };
+      auto wait = [&](uint64_t* bar, uint32_t par) -> bool {
+        if (!mbar_wait_or_abort(bar, par, &bars->abort_flag)) {
+          raise_abort(bars, p.err, kErrMma);
+          ok = false;
+          return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      for (int g = pair; g < p.total && ok; g += npairs) {
+        const Item it = decode_item(p, g);
+        const bool active = t < it.nslots;
+        if (active) {
+          if (!wait(&bars->q_full[t], q_cnt & 1)) break;
+          ++q_cnt;
+          // S of the first two K/V tiles (both S buffers)
+          const int pre = it.nkv < 2 ? it.nkv : 2;
+          for (int jj = 0; jj < pre; ++jj) {
+            const uint32_t idx = kv_base + jj, st = idx % kStages;
+            if (!wait(&bars->kv_full[st], (idx / kStages) & 1)) break;
+            issue_s(st);
+            if (jj == it.nkv - 1) commit_pair(&bars->q_empty[t]);
+          }
+          if (!ok) break;
+        }
+        // per K/V tile j: P V_j as soon as P is written, then S of tile j + 2 into the buffer
+        // that P V_j reads (one thread's MMAs run in issue order); then release stage j
+        for (int j = 0; j < it.nkv; ++j) {
+          const uint32_t idx = kv_base + j, st = idx % kStages;
+          if (active) {
+            // the K/V stage of tile j + 2 first (normally long full), so that PV_j and S_{j+2}
+            // go out back to back as soon as P_j is written
+            const bool more = j + 2 < it.nkv;
+            const uint32_t idx2 = idx + 2, st2 = idx2 % kStages;
+            if (more && !wait(&bars->kv_full[st2], (idx2 / kStages) & 1)) break;
+            if (!wait(&bars->p_full[t][p_seq & 1], (p_seq >> 1) & 1)) break;
+            issue_pv(st, j > 0 ? 1u : 0u);
+            if (more) {
+              issue_s(st2);
+              if (j + 3 == it.nkv) commit_pair(&bars->q_empty[t]);
+            }
+          } else {
+            if (!wait(&bars->kv_full[st], (idx / kStages) & 1)) break;
+          }
+          commit_pair(&bars->kv_empty[st]);
+        }
+        kv_base += it.nkv;
+      }
+      // every MMA this thread issued completes before either CTA can release TMEM or leave
+      commit_pair(&bars->drain[t]);
+      mbar_wait(&bars->drain[t], 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue (both CTAs)
+    regs_alloc<kHighRegs>();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
+    const int t = (warp - 4) >> 2;  // slot of this warpgroup
+    const int wl = warp & 3;        // TMEM lane quarter
+    const int row = wl * 32 + lane; // row inside this CTA's 128-row tile
+    const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + t * 128;
+    const uint32_t t_o = tmem + lane_off + 256 + t * 128;
+    const uint32_t p_full_l = map_to(&bars->p_full[t][0], 0);  // the leader's P barriers of this slot
+    uint32_t seq = 0;
+    // wait until the P V MMA of sequence number n (and every earlier one) is complete; when this
+    // is called the one of n - 2 is known to be complete, so the buffer's barrier is at most one
+    // phase short of the one awaited
+    auto pv_done = [&](uint32_t n) { return warp_wait(bars, &bars->o_done[t][n & 1], (n >> 1) & 1, p.err); };
+    bool ok = true;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+    for (int g = pair; g < p.total && ok; g += npairs) {
+      const Item it = decode_item(p, g);
+      if (t >= it.nslots) continue;
+      float m = -FLT_MAX, l = 0.f;
+      for (int j = 0; j < it.nkv; ++j, ++seq) {
+        const uint32_t buf = t_s + (seq & 1) * kBN;
+        if (!warp_wait(bars, &bars->s_full[t][seq & 1], (seq >> 1) & 1, p.err)) { ok = false; break; }
+        uint32_t r[kCols];
+        tmem_ld32(buf, r);
+        tmem_ld32(buf + 32, r + 32);
+        tmem_ld_wait<kCols>(r);
+        if (j == it.nkv - 1 && it.last_valid < kBN) {  // ragged last K/V tile (uniform branch)
+#pragma unroll
+          for (int i = 0; i < kCols; ++i)
+            if (i >= it.last_valid) r[i] = __float_as_uint(-INFINITY);
+        }
+        // row max: 8 independent chains of 3-input max over the 64 scores
+        float mc[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          mc[c] = fmax3(__uint_as_float(r[c]), __uint_as_float(r[8 + c]), __uint_as_float(r[16 + c]));
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[24 + c]), __uint_as_float(r[32 + c]));
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[40 + c]), __uint_as_float(r[48 + c]));
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mc[c] = fmaxf(mc[c], __uint_as_float(r[56 + c]));
+        const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7])) *
+                         p.scale_log2;
+        const bool need = (j > 0) && (mx > m + kRescaleThreshold);
+        const float alpha = need ? ex2_approx(m - mx) : 1.0f;
+        if (j == 0 || need) m = mx;
+        if (__any_sync(0xffffffffu, need)) {
+          if (!pv_done(seq - 1)) { ok = false; break; }
+#pragma unroll 1
+          for (int c = 0; c < kD / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + 32 * c, o);
+            tmem_ld_wait<32>(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_o + 32 * c, o);
+          }
+        }
+        // p = 2^(s * scale - m) in pairs, written over this tile's S buffer as bf16 pairs
+        const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(-m, -m);
+        uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < kCols / 2; ++i) {
+          const uint64_t x =
+              ffma2(static_cast<uint64_t>(r[2 * i]) | (static_cast<uint64_t>(r[2 * i + 1]) << 32), sc2, nm2);
+          const uint64_t e = (i % kPolyDen < kPolyNum) ? exp2_poly2(x) : pack2(ex2_approx(lo2(x)), ex2_approx(hi2(x)));
+          acc[i & 3] = fadd2(acc[i & 3], e);
+          __nv_bfloat162 hv = __floats2bfloat162_rn(lo2(e), hi2(e));
+          r[i] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+        tmem_st32(buf, r);
+        tmem_st_wait();
+        tc_fence_before();
+        arrive_cluster(p_full_l + 8u * (seq & 1));
+        const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+        l = l * alpha + (lo2(a2) + hi2(a2));
+      }
+      if (!ok) break;
+      // epilogue: O / l at the row's original token position
+      const float inv_l = 1.0f / l;
+      if (!pv_done(seq - 1)) { ok = false; break; }
+      const int ut = 2 * t + (int)rank;
+      const int u = ut * p.bpt + row / p.b;
+      const bool store = (ut < it.ntiles) && (u < it.nblk);
+      const size_t token = (size_t)it.blk(store ? u : 0) * p.b + (row % p.b);
+      __nv_bfloat16* dst = out + ((size_t)it.bh * p.N + token) * kD;
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + 32 * c, o);
+        tmem_ld_wait<32>(o);
+        float* f = reinterpret_cast<float*>(o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(o[i]) * inv_l;
+        if (store) store_row_chunk(dst + 32 * c, f);
+      }
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_warp();  // both CTAs done with TMEM, shared memory and the leader's barriers
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(
+                     *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base)),
+                 "r"(512)
+                 : "memory");
+  }
+}
+
+}  // namespace
+
+bool attention_pair_supported(const Plan& p) { return p.dt == 0 && p.D == kD; }
+
+cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, void* out, const Plan& pl,
+                                  const Work& w, cudaStream_t s, int* n_ctas) {
+  PairParams p{};
+  p.route = w.route;
+  p.out = out;
+  p.err = w.ctrl;
+  p.BH = pl.BH;
+  p.N = pl.N;
+  p.b = pl.b;
+  p.L_src = pl.L_src;
+  p.n_q = pl.n_q;
+  p.n_exact = pl.n_exact;
+  p.n_flat = pl.n_flat;
+  p.L_new = pl.L_new;
+  p.n_new = pl.n_new;
+  p.bpt = kBM / pl.b;
+  p.bpi = 4 * p.bpt;
+  p.items_e = (pl.n_exact + p.bpi - 1) / p.bpi;
+  p.items_t = (pl.n_flat + p.bpi - 1) / p.bpi;
+  p.total = pl.BH * (p.items_e + p.items_t);
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+  if (n_ctas) *n_ctas = 0;
+  if (p.total == 0) return cudaSuccess;
+
+  CUtensorMap tq, tk, tks, tv, tvs, tkc, tvc;
+  const bool has_sel = pl.k > 0;
+  const int sel_rows = has_sel ? pl.k * pl.b : pl.N;
+  const bool ok = make_map(&tq, q, 2, kD, pl.N, pl.BH, 64) && make_map(&tk, k, 2, kD, pl.N, pl.BH, kKRows) &&
+                  make_map(&tks, has_sel ? w.ksel : k, 2, kD, sel_rows, pl.BH, kKRows) &&
+                  make_map(&tkc, w.kcn, 2, kD, pl.n_new, pl.BH, kKRows) &&
+                  make_map(&tv, v, 2, kD, pl.N, pl.BH, kBN) &&
+                  make_map(&tvs, has_sel ? w.vsel : v, 2, kD, sel_rows, pl.BH, kBN) &&
+                  make_map(&tvc, w.vcn, 2, kD, pl.n_new, pl.BH, kBN);
+  if (!ok) return cudaErrorInvalidValue;
+
+  auto kern = attention_pair_kernel;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // the register split needs this count
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+  if (e != cudaSuccess) return e;
+  // as many CTA pairs as can be resident at once (one CTA per SM), at most one per work item
+  static int cached_pairs[64] = {0};
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  int pairs = dev >= 0 && dev < 64 ? cached_pairs[dev] : 0;
+  if (pairs <= 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemAlloc;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg)) != cudaSuccess) return e;
+    if (pairs <= 0) return cudaErrorLaunchOutOfResources;
+    if (dev >= 0 && dev < 64) cached_pairs[dev] = pairs;
+  }
+  if (pairs > p.total) pairs = p.total;
+  kern<<<2 * pairs, kThreads, kSmemAlloc, s>>>(tq, tk, tks, tv, tvs, tkc, tvc, p);
+  if (n_ctas) *n_ctas = 2 * pairs;
+  return cudaGetLastError();
+}
+
+}  // namespace isa

@@ -61,6 +61,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Like mbar_wait, but also gives up (returning false) once *abort is set. The flag is
+// read only when the phase is not already complete: on the fast path this costs one
+// try_wait, which matters on threads that issue tensor-core work between waits.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, const int* abort,
+                                                   uint64_t timeout_ns = kWaitTimeoutNs) {
+  const uint32_t a = smem_addr(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(a, parity)) return true;
+    if (*reinterpret_cast<const volatile int*>(abort) != 0) return false;
+    if (global_timer_ns() - t0 > timeout_ns) return false;
+  }
+}
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
