@@ -64,6 +64,14 @@ def hbm_bytes_per_call(w) -> dict:
     return dict(pool=3.0 * w.B * w.H * N * w.D * e, gather=2.0 * 2.0 * w.B * w.H * k * w.b * w.D * e)
 
 
+def attention_source_sha1(w) -> str:
+    """sha1 of the attention kernel source this workload runs on (CTA pairs for bf16 D=128)."""
+    import hashlib
+    name = "k_attention_pair.cu" if (w.dtype == "bf16" and w.D == 128) else "k_attention.cu"
+    with open(os.path.join(ROOT, "block_sparse_attention_isa_b200", "csrc", name), "rb") as fh:
+        return hashlib.sha1(fh.read()).hexdigest()
+
+
 def reduce_max(x: float, dist=None) -> float:
     """Max of a float over all ranks (identity without a process group)."""
     if dist is None or not dist.is_initialized():
@@ -295,7 +303,10 @@ def run_ours(args, w):
     prof = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(prof):
         with open(prof) as fh:
-            traffic = json.load(fh).get(w.name, {}).get("attention")
+            ent = json.load(fh).get(w.name, {})
+        # the counters hold only for the kernel source they were taken on
+        if ent.get("kernel_source_sha1") == attention_source_sha1(w):
+            traffic = ent.get("attention")
 
     # end to end through the host-buffer entry point (pinned host memory, copies inside the timed region)
     e2e = None

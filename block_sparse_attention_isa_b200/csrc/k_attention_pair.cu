@@ -177,6 +177,20 @@ __device__ __forceinline__ void mma_ts_pair(uint32_t d, uint32_t a_tmem, uint32_
       : "memory");
 }
 
+// The k-th work item of CTA pair `pair`, or -1 past its last. Exact items all cost the same
+// and go round-robin over the pairs; when they do not divide evenly, the first E % npairs
+// pairs hold one more of them, so the (much cheaper) Taylor items go round-robin over the
+// other pairs only. Every role of both CTAs walks the same sequence.
+__device__ __forceinline__ int schedule(const PairParams& p, int pair, int npairs, int k) {
+  const int E = p.BH * p.items_e, T = p.BH * p.items_t;
+  const int n_exact = pair < E ? (E - pair + npairs - 1) / npairs : 0;
+  if (k < n_exact) return pair + k * npairs;
+  const int busy = E % npairs;
+  if (pair < busy) return -1;
+  const int g = (pair - busy) + (k - n_exact) * (npairs - busy);
+  return g < T ? E + g : -1;
+}
+
 struct Item {
   int bh, kind, nblk, ntiles, nslots, nkv, last_valid;
   const int32_t* lst;
@@ -301,7 +315,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t kv_full_l = map_to(&bars->kv_full[0], 0);
       uint32_t kv_it = 0, q_loads0 = 0, q_loads1 = 0;
       bool ok = true;
-      for (int g = pair; g < p.total && ok; g += npairs) {
+      for (int k = 0, g = schedule(p, pair, npairs, 0); g >= 0 && ok; g = schedule(p, pair, npairs, ++k)) {
         const Item it = decode_item(p, g);
         for (int t = 0; t < it.nslots; ++t) {
           // slot t's Q buffer is free once the S MMAs of the last item that used it are complete
@@ -423,7 +437,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         return true;
       };
-      for (int g = pair; g < p.total && ok; g += npairs) {
+      for (int k = 0, g = schedule(p, pair, npairs, 0); g >= 0 && ok; g = schedule(p, pair, npairs, ++k)) {
         const Item it = decode_item(p, g);
         const bool active = t < it.nslots;
         if (active) {
@@ -485,7 +499,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto pv_done = [&](uint32_t n) { return warp_wait(bars, &bars->o_done[t][n & 1], (n >> 1) & 1, p.err); };
     bool ok = true;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-    for (int g = pair; g < p.total && ok; g += npairs) {
+    for (int k = 0, g = schedule(p, pair, npairs, 0); g >= 0 && ok; g = schedule(p, pair, npairs, ++k)) {
       const Item it = decode_item(p, g);
       if (t >= it.nslots) continue;
       float m = -FLT_MAX, l = 0.f;
