@@ -20,7 +20,8 @@
 //    words, conflict-free shared-memory reads);
 //  * a grid barrier (all block means written);
 //  * phase 2: scoring items (head, 16 source rows) are dealt round-robin; each
-//    computes its rows of S_coarse (CUDA cores, fp32), their softmax, and the
+//    computes its rows of S_coarse (CUDA cores, fp32; the key blocks pass
+//    through shared memory in chunks of 64), their softmax, and the
 //    rows' sum on every context column, written as a partial. The last item of
 //    a head to finish adds the partials in a fixed order (deterministic), then
 //    runs the top-k as a shared-memory bitonic sort.
@@ -37,6 +38,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kRows = 16;                  // source query blocks per scoring item
+constexpr int kKeys = 64;                  // pooled key blocks per shared-memory chunk in phase 2
+constexpr int kGroups = kThreads / kKeys;  // phase-2 row groups (kRows / kGroups rows per thread)
+static_assert(kRows % kGroups == 0, "rows per group");
 constexpr int kStageBudget = 192 * 1024;   // shared memory for the phase-1 ring
 constexpr int kMaxStages = 8;
 
@@ -56,7 +60,7 @@ struct PoolCfg {
 
 int score_scratch_floats(const Plan& p, int D) {
   const int P = next_pow2(p.n_ctx < 1 ? 1 : p.n_ctx);
-  return kRows * D + kRows * p.n_q + p.n_ctx + 2 * P + next_pow2(p.k < 1 ? 1 : p.k);
+  return kRows * D + kKeys * (D + 4) + kRows * p.n_q + p.n_ctx + 2 * P + next_pow2(p.k < 1 ? 1 : p.k);
 }
 
 template <typename T>
@@ -182,8 +186,10 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
   // ---- phase 2: coarse scores, context-column partial sums, top-k ----------------------
   const int n_q = p.n_q, n_src = p.n_src, n_ctx = p.n_ctx;
   const int n_chunks = (n_src + kRows - 1) / kRows;
+  constexpr int KS = D + 4;                         // key row stride: 4-word skew between rows
   float* qcs = reinterpret_cast<float*>(smem);      // [kRows][D]
-  float* lg = qcs + kRows * D;                      // [kRows][n_q]
+  float* ks = qcs + kRows * D;                      // [kKeys][KS]
+  float* lg = ks + kKeys * KS;                      // [kRows][n_q]
   float* cs = lg + kRows * n_q;                     // [n_ctx]
   const int P = next_pow2(n_ctx < 1 ? 1 : n_ctx);
   float* skey = cs + n_ctx;                         // [P]
@@ -198,31 +204,47 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
     const float* Qc = w.qc + (size_t)bh * n_q * D;
     const float* Kc = w.kc + (size_t)bh * n_q * D;
     __syncthreads();
-    for (int e = tid; e < kRows * D; e += kThreads) {
-      const int r = e / D;
-      qcs[e] = r < nr ? __ldcg(Qc + (size_t)(i0 + r) * D + (e - r * D)) : 0.f;
+    for (int e = tid; e < kRows * (D / 4); e += kThreads) {
+      const int r = e / (D / 4), d4 = e - r * (D / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < nr) v = __ldcg(reinterpret_cast<const float4*>(Qc + (size_t)(i0 + r) * D) + d4);
+      *reinterpret_cast<float4*>(qcs + r * D + 4 * d4) = v;
     }
-    __syncthreads();
-    for (int j = tid; j < n_q; j += kThreads) {
-      float a[kRows];
+    // the key blocks pass through shared memory in chunks of kKeys (coalesced loads); thread
+    // (key kk, row group rg) accumulates kRows / kGroups scores, summing over d in order
+    constexpr int RPG = kRows / kGroups;
+    const int kj = tid % kKeys, rg = tid / kKeys;
+    for (int j0 = 0; j0 < n_q; j0 += kKeys) {
+      __syncthreads();
+      for (int e = tid; e < kKeys * (D / 4); e += kThreads) {
+        const int jj = e / (D / 4), d4 = e - jj * (D / 4);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j0 + jj < n_q) v = __ldcg(reinterpret_cast<const float4*>(Kc + (size_t)(j0 + jj) * D) + d4);
+        *reinterpret_cast<float4*>(ks + jj * KS + 4 * d4) = v;
+      }
+      __syncthreads();
+      float a[RPG];
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) a[r] = 0.f;
-      const float4* kr = reinterpret_cast<const float4*>(Kc + (size_t)j * D);
-#pragma unroll 2
+      for (int r = 0; r < RPG; ++r) a[r] = 0.f;
+      const float* kr = ks + kj * KS;
+#pragma unroll 4
       for (int d4 = 0; d4 < D / 4; ++d4) {
-        const float4 kv = __ldcg(kr + d4);
+        const float4 kv = *reinterpret_cast<const float4*>(kr + 4 * d4);
 #pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-          const float4 qv = *reinterpret_cast<const float4*>(qcs + r * D + 4 * d4);
+        for (int r = 0; r < RPG; ++r) {
+          const float4 qv = *reinterpret_cast<const float4*>(qcs + (rg * RPG + r) * D + 4 * d4);
           a[r] = fmaf(qv.x, kv.x, a[r]);
           a[r] = fmaf(qv.y, kv.y, a[r]);
           a[r] = fmaf(qv.z, kv.z, a[r]);
           a[r] = fmaf(qv.w, kv.w, a[r]);
         }
       }
+      const int j = j0 + kj;
+      if (j < n_q) {
 #pragma unroll
-      for (int r = 0; r < kRows; ++r)
-        if (r < nr) lg[r * n_q + j] = a[r] * scale;
+        for (int r = 0; r < RPG; ++r)
+          if (rg * RPG + r < nr) lg[(rg * RPG + r) * n_q + j] = a[r] * scale;
+      }
     }
     __syncthreads();
     for (int r = warp; r < nr; r += kThreads / 32) {  // row softmax, one warp per row

@@ -12,11 +12,14 @@
 // free of the cancellation of sum p^2/n - 1/n^2), and the n_flat blocks of
 // LOWEST sharpness (ties by lower index) take the Taylor path.
 //
-// Grid (ceil(n_q / 8), B*H), 256 threads. Each CTA scores 8 query blocks
-// against all n_new pooled key blocks and writes their M_i; it also writes
-// its share of the pooled K_new / V_new rows in the attention kernel's element
-// type. The last CTA of a head sorts (M_i, i), then writes the route list:
-// exact blocks ascending followed by Taylor blocks ascending.
+// Grid (ceil(n_q / R), B*H), 256 threads, R = 32 query blocks per CTA (16 when
+// n_new is above 1024). The CTA keeps its R pooled query rows in shared memory
+// and streams the gathered pooled keys of K_new through shared memory in
+// chunks of 64 (rows padded so that the 32 keys a warp reads fall in distinct
+// banks); thread (key, row group) accumulates R / 4 scores. It writes the M_i of
+// its rows, and its share of the pooled K_new / V_new rows in the attention
+// kernel's element type. The last CTA of a head sorts (M_i, i), then writes the
+// route list: exact blocks ascending followed by Taylor blocks ascending.
 #include <cuda_bf16.h>
 #include <float.h>
 
@@ -27,53 +30,77 @@ namespace isa {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kRows = 8;  // query blocks per CTA
+constexpr int kKeys = 64;     // pooled keys per shared-memory chunk
+constexpr int kGroups = kThreads / kKeys;  // row groups
 
 __device__ __forceinline__ void store_elem(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void store_elem(float* p, float x) { *p = x; }
 
-template <typename T, int D>
+template <int D>
+__host__ __device__ constexpr int key_stride() { return D + 4; }  // floats; 4-word skew between consecutive key rows
+
+template <typename T, int D, int R>
 __global__ void __launch_bounds__(kThreads) route_kernel(Plan p, Work w) {
+  constexpr int KS = key_stride<D>();
+  constexpr int RPG = R / kGroups;  // rows per thread
+  static_assert(R % kGroups == 0, "rows per group");
   extern __shared__ __align__(16) float smem[];
-  const int bh = blockIdx.y, i0 = blockIdx.x * kRows, tid = threadIdx.x;
+  const int bh = blockIdx.y, i0 = blockIdx.x * R, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int n_q = p.n_q, n_src = p.n_src, n_new = p.n_new;
-  const int nr = min(kRows, n_q - i0);
+  const int nr = min(R, n_q - i0);
   const float* Qc = w.qc + (size_t)bh * n_q * D;
   const float* Kc = w.kc + (size_t)bh * n_q * D;
   const float* Vc = w.vc + (size_t)bh * n_q * D;
   const int32_t* sel = w.sel + (size_t)bh * p.k;
-  float* qcs = smem;                 // [kRows][D]
-  float* lg = qcs + kRows * D;       // [kRows][n_new]
+  float* qs = smem;              // [R][D]
+  float* ks = qs + R * D;        // [kKeys][KS]
+  float* lg = ks + kKeys * KS;   // [R][n_new]
   __shared__ int s_last;
 
-  for (int e = tid; e < kRows * D; e += kThreads) {
-    const int r = e / D;
-    qcs[e] = r < nr ? Qc[(size_t)(i0 + r) * D + (e % D)] : 0.f;
+  for (int e = tid; e < R * (D / 4); e += kThreads) {
+    const int r = e / (D / 4), d4 = e - r * (D / 4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < nr) v = __ldcg(reinterpret_cast<const float4*>(Qc + (size_t)(i0 + r) * D) + d4);
+    *reinterpret_cast<float4*>(qs + r * D + 4 * d4) = v;
   }
-  __syncthreads();
   const float scale = 1.0f / sqrtf((float)D);
-  for (int j = tid; j < n_new; j += kThreads) {
-    const int src = j < n_src ? j : n_src + sel[j - n_src];
-    const float4* kr = reinterpret_cast<const float4*>(Kc + (size_t)src * D);
-    float a[kRows];
+  const int kk = tid % kKeys, rg = tid / kKeys;
+  for (int j0 = 0; j0 < n_new; j0 += kKeys) {
+    __syncthreads();  // the previous chunk is consumed (and the query rows are in place)
+    for (int e = tid; e < kKeys * (D / 4); e += kThreads) {
+      const int jj = e / (D / 4), d4 = e - jj * (D / 4);
+      const int j = j0 + jj;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < n_new) {
+        const int src = j < n_src ? j : n_src + sel[j - n_src];
+        v = __ldcg(reinterpret_cast<const float4*>(Kc + (size_t)src * D) + d4);
+      }
+      *reinterpret_cast<float4*>(ks + jj * KS + 4 * d4) = v;
+    }
+    __syncthreads();
+    float a[RPG];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) a[r] = 0.f;
+    for (int r = 0; r < RPG; ++r) a[r] = 0.f;
+    const float* kr = ks + kk * KS;
 #pragma unroll 4
     for (int d4 = 0; d4 < D / 4; ++d4) {
-      const float4 kv = kr[d4];
+      const float4 kv = *reinterpret_cast<const float4*>(kr + 4 * d4);
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        const float4 qv = *reinterpret_cast<const float4*>(qcs + r * D + 4 * d4);
+      for (int r = 0; r < RPG; ++r) {
+        const float4 qv = *reinterpret_cast<const float4*>(qs + (rg * RPG + r) * D + 4 * d4);
         a[r] = fmaf(qv.x, kv.x, a[r]);
         a[r] = fmaf(qv.y, kv.y, a[r]);
         a[r] = fmaf(qv.z, kv.z, a[r]);
         a[r] = fmaf(qv.w, kv.w, a[r]);
       }
     }
+    const int j = j0 + kk;
+    if (j < n_new) {
 #pragma unroll
-    for (int r = 0; r < kRows; ++r)
-      if (r < nr) lg[r * n_new + j] = a[r] * scale;
+      for (int r = 0; r < RPG; ++r)
+        if (rg * RPG + r < nr) lg[(rg * RPG + r) * n_new + j] = a[r] * scale;
+    }
   }
   __syncthreads();
   const float inv_n = 1.0f / (float)n_new;
@@ -101,12 +128,11 @@ __global__ void __launch_bounds__(kThreads) route_kernel(Plan p, Work w) {
   // pooled K_new / V_new rows for the Taylor path, in the MMA element type
   T* kcn = static_cast<T*>(w.kcn) + (size_t)bh * n_new * D;
   T* vcn = static_cast<T*>(w.vcn) + (size_t)bh * n_new * D;
-  for (int j = blockIdx.x; j < n_new; j += gridDim.x) {
+  for (int e = tid + blockIdx.x * kThreads; e < n_new * D; e += gridDim.x * kThreads) {
+    const int j = e / D, d = e - j * D;
     const int src = j < n_src ? j : n_src + sel[j - n_src];
-    for (int d = tid; d < D; d += kThreads) {
-      store_elem(kcn + (size_t)j * D + d, Kc[(size_t)src * D + d]);
-      store_elem(vcn + (size_t)j * D + d, Vc[(size_t)src * D + d]);
-    }
+    store_elem(kcn + e, Kc[(size_t)src * D + d]);
+    store_elem(vcn + e, Vc[(size_t)src * D + d]);
   }
 
   __threadfence();
@@ -143,20 +169,26 @@ __global__ void __launch_bounds__(kThreads) route_kernel(Plan p, Work w) {
   }
 }
 
-template <typename T, int D>
-cudaError_t launch_t(const Plan& p, const Work& w, cudaStream_t s) {
+template <typename T, int D, int R>
+cudaError_t launch_r(const Plan& p, const Work& w, cudaStream_t s) {
   const int P = next_pow2(p.n_q);
-  size_t a = sizeof(float) * (size_t)(kRows * D + kRows * p.n_new);
-  size_t b = (sizeof(float) + 2 * sizeof(int32_t)) * (size_t)P;
+  const size_t a = sizeof(float) * (size_t)(R * D + kKeys * key_stride<D>() + R * p.n_new);
+  const size_t b = (sizeof(float) + 2 * sizeof(int32_t)) * (size_t)P;
   const size_t smem = a > b ? a : b;
-  auto kern = route_kernel<T, D>;
+  auto kern = route_kernel<T, D, R>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid((p.n_q + kRows - 1) / kRows, p.BH);
+  dim3 grid((p.n_q + R - 1) / R, p.BH);
   kern<<<grid, kThreads, smem, s>>>(p, w);
   return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const Plan& p, const Work& w, cudaStream_t s) {
+  // 32 query blocks per CTA; 16 when the scores of 32 rows would not fit in shared memory
+  return p.n_new <= 1024 ? launch_r<T, D, 32>(p, w, s) : launch_r<T, D, 16>(p, w, s);
 }
 
 }  // namespace
