@@ -19,9 +19,10 @@
 //    are in flight per SM while the previous one is reduced (fp32 sums, 4-byte
 //    words, conflict-free shared-memory reads);
 //  * a grid barrier (all block means written);
-//  * phase 2: scoring items (head, 16 source rows) are dealt round-robin; each
-//    computes its rows of S_coarse (CUDA cores, fp32; the key blocks pass
-//    through shared memory in chunks of 64), their softmax, and the
+//  * phase 2: scoring items (head, 48 source rows, or 16 when n_q > 512) are
+//    dealt round-robin; each computes its rows of S_coarse (CUDA cores, fp32;
+//    the key blocks pass through shared memory in double-buffered chunks of
+//    64), their softmax, and the
 //    rows' sum on every context column, written as a partial. The last item of
 //    a head to finish adds the partials in a fixed order (deterministic), then
 //    runs the top-k as a shared-memory bitonic sort.
@@ -36,11 +37,25 @@
 namespace isa {
 namespace {
 
+// 16-byte global -> shared copies that complete asynchronously (groups committed and awaited).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int n>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory"); }
+
 constexpr int kThreads = 256;
-constexpr int kRows = 16;                  // source query blocks per scoring item
 constexpr int kKeys = 64;                  // pooled key blocks per shared-memory chunk in phase 2
-constexpr int kGroups = kThreads / kKeys;  // phase-2 row groups (kRows / kGroups rows per thread)
-static_assert(kRows % kGroups == 0, "rows per group");
+constexpr int kGroups = kThreads / kKeys;  // phase-2 row groups (R / kGroups rows per thread)
+// Source query blocks per scoring item: 48 (three items per head at the 32K-token workload, so
+// all items run in one round) while the item's scores, 48 x n_q floats, fit in shared memory;
+// 16 above that.
+constexpr int kRowsLarge = 48;
+constexpr int kRowsSmall = 16;
+constexpr int kLargeMaxNq = 512;
+static_assert(kRowsLarge % kGroups == 0 && kRowsSmall % kGroups == 0, "rows per group");
+inline int rows_per_item(int n_q) { return n_q <= kLargeMaxNq ? kRowsLarge : kRowsSmall; }
 constexpr int kStageBudget = 192 * 1024;   // shared memory for the phase-1 ring
 constexpr int kMaxStages = 8;
 
@@ -58,9 +73,9 @@ struct PoolCfg {
   static_assert(STAGES >= 2, "at least two stages");
 };
 
-int score_scratch_floats(const Plan& p, int D) {
+int score_scratch_floats(const Plan& p, int D, int R) {
   const int P = next_pow2(p.n_ctx < 1 ? 1 : p.n_ctx);
-  return kRows * D + kKeys * (D + 4) + kRows * p.n_q + p.n_ctx + 2 * P + next_pow2(p.k < 1 ? 1 : p.k);
+  return R * D + 2 * kKeys * (D + 4) + R * p.n_q + p.n_ctx + 2 * P + next_pow2(p.k < 1 ? 1 : p.k);
 }
 
 template <typename T>
@@ -101,7 +116,7 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t* err) {
   return s_ok != 0;
 }
 
-template <typename T, int D, int BLK>
+template <typename T, int D, int BLK, int R>
 __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                                       const T* __restrict__ v, Plan p, Work w) {
   using C = PoolCfg<T, D, BLK>;
@@ -185,12 +200,12 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
 
   // ---- phase 2: coarse scores, context-column partial sums, top-k ----------------------
   const int n_q = p.n_q, n_src = p.n_src, n_ctx = p.n_ctx;
-  const int n_chunks = (n_src + kRows - 1) / kRows;
+  const int n_chunks = (n_src + R - 1) / R;
   constexpr int KS = D + 4;                         // key row stride: 4-word skew between rows
-  float* qcs = reinterpret_cast<float*>(smem);      // [kRows][D]
-  float* ks = qcs + kRows * D;                      // [kKeys][KS]
-  float* lg = ks + kKeys * KS;                      // [kRows][n_q]
-  float* cs = lg + kRows * n_q;                     // [n_ctx]
+  float* qcs = reinterpret_cast<float*>(smem);      // [R][D]
+  float* ks = qcs + R * D;                          // [2][kKeys][KS]: double-buffered key chunks
+  float* lg = ks + 2 * kKeys * KS;                  // [R][n_q]
+  float* cs = lg + R * n_q;                         // [n_ctx]
   const int P = next_pow2(n_ctx < 1 ? 1 : n_ctx);
   float* skey = cs + n_ctx;                         // [P]
   int32_t* sidx = reinterpret_cast<int32_t*>(skey + P);
@@ -200,33 +215,44 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
   __shared__ int s_last;
   for (int item = g; item < p.BH * n_chunks; item += G) {
     const int bh = item / n_chunks, chunk = item - bh * n_chunks;
-    const int i0 = chunk * kRows, nr = min(kRows, n_src - i0);
+    const int i0 = chunk * R, nr = min(R, n_src - i0);
     const float* Qc = w.qc + (size_t)bh * n_q * D;
     const float* Kc = w.kc + (size_t)bh * n_q * D;
     __syncthreads();
-    for (int e = tid; e < kRows * (D / 4); e += kThreads) {
+    for (int e = tid; e < R * (D / 4); e += kThreads) {
       const int r = e / (D / 4), d4 = e - r * (D / 4);
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (r < nr) v = __ldcg(reinterpret_cast<const float4*>(Qc + (size_t)(i0 + r) * D) + d4);
       *reinterpret_cast<float4*>(qcs + r * D + 4 * d4) = v;
     }
-    // the key blocks pass through shared memory in chunks of kKeys (coalesced loads); thread
-    // (key kk, row group rg) accumulates kRows / kGroups scores, summing over d in order
-    constexpr int RPG = kRows / kGroups;
+    // the key blocks pass through shared memory in chunks of kKeys, double-buffered: the next
+    // chunk is copied (cp.async, 16 bytes a thread at a time) while this one is scored; thread
+    // (key kj, row group rg) accumulates R / kGroups scores, summing over d in order
+    constexpr int RPG = R / kGroups;
     const int kj = tid % kKeys, rg = tid / kKeys;
-    for (int j0 = 0; j0 < n_q; j0 += kKeys) {
-      __syncthreads();
+    const int n_kc = (n_q + kKeys - 1) / kKeys;
+    auto stage_chunk = [&](int c) {
+      float* dstb = ks + (c & 1) * kKeys * KS;
+      const int j0 = c * kKeys;
       for (int e = tid; e < kKeys * (D / 4); e += kThreads) {
         const int jj = e / (D / 4), d4 = e - jj * (D / 4);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (j0 + jj < n_q) v = __ldcg(reinterpret_cast<const float4*>(Kc + (size_t)(j0 + jj) * D) + d4);
-        *reinterpret_cast<float4*>(ks + jj * KS + 4 * d4) = v;
+        if (j0 + jj < n_q) cp_async16(dstb + jj * KS + 4 * d4, Kc + (size_t)(j0 + jj) * D + 4 * d4);
       }
-      __syncthreads();
+      cp_async_commit();
+    };
+    stage_chunk(0);
+    for (int c = 0; c < n_kc; ++c) {
+      if (c + 1 < n_kc) {
+        stage_chunk(c + 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();  // chunk c (and, the first time, the query rows) visible to every thread
       float a[RPG];
 #pragma unroll
       for (int r = 0; r < RPG; ++r) a[r] = 0.f;
-      const float* kr = ks + kj * KS;
+      const float* kr = ks + (c & 1) * kKeys * KS + kj * KS;
 #pragma unroll 4
       for (int d4 = 0; d4 < D / 4; ++d4) {
         const float4 kv = *reinterpret_cast<const float4*>(kr + 4 * d4);
@@ -239,14 +265,14 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
           a[r] = fmaf(qv.w, kv.w, a[r]);
         }
       }
-      const int j = j0 + kj;
+      const int j = c * kKeys + kj;
       if (j < n_q) {
 #pragma unroll
         for (int r = 0; r < RPG; ++r)
           if (rg * RPG + r < nr) lg[(rg * RPG + r) * n_q + j] = a[r] * scale;
       }
+      __syncthreads();  // chunk c consumed: its buffer is refilled with chunk c + 2 next round
     }
-    __syncthreads();
     for (int r = warp; r < nr; r += kThreads / 32) {  // row softmax, one warp per row
       float* row = lg + r * n_q;
       float m = -FLT_MAX;
@@ -300,13 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
   }
 }
 
-template <typename T, int D, int BLK>
-cudaError_t launch_t(const void* q, const void* k, const void* v, const Plan& p, const Work& w, cudaStream_t s) {
+template <typename T, int D, int BLK, int R>
+cudaError_t launch_r(const void* q, const void* k, const void* v, const Plan& p, const Work& w, cudaStream_t s) {
   using C = PoolCfg<T, D, BLK>;
   const size_t ring = (size_t)C::STAGES * C::STAGE_BYTES + sizeof(uint64_t) * kMaxStages + sizeof(float) * C::RED_FLOATS;
-  const size_t score = sizeof(float) * (size_t)score_scratch_floats(p, D);
+  const size_t score = sizeof(float) * (size_t)score_scratch_floats(p, D, R);
   const size_t smem = ring > score ? ring : score;
-  auto kern = pool_score_topk_kernel<T, D, BLK>;
+  auto kern = pool_score_topk_kernel<T, D, BLK, R>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -324,10 +350,17 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, const Plan& p,
   return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kern), dim3(grid), dim3(kThreads), args, smem, s);
 }
 
+template <typename T, int D, int BLK>
+cudaError_t launch_t(const void* q, const void* k, const void* v, const Plan& p, const Work& w, cudaStream_t s) {
+  return rows_per_item(p.n_q) == kRowsLarge ? launch_r<T, D, BLK, kRowsLarge>(q, k, v, p, w, s)
+                                            : launch_r<T, D, BLK, kRowsSmall>(q, k, v, p, w, s);
+}
+
 }  // namespace
 
 size_t pool_partial_floats(const Plan& p) {
-  return (size_t)p.BH * ((p.n_src + kRows - 1) / kRows) * p.n_ctx;
+  const int R = rows_per_item(p.n_q);
+  return (size_t)p.BH * ((p.n_src + R - 1) / R) * p.n_ctx;
 }
 
 cudaError_t launch_pool_score_topk(const void* q, const void* k, const void* v, const Plan& p, const Work& w,

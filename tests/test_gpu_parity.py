@@ -157,3 +157,28 @@ def test_polynomial_exp2_against_cuda_exp2f():
     assert rel <= 1e-4, rel
     exact = torch.from_numpy(np.exp2(x.cpu().double().numpy()))
     assert ((yp.cpu().double() - exact).abs() / exact).max().item() <= 1e-4
+
+
+def test_many_query_blocks_scoring_path():
+    """n_q = 640 query blocks (above 512, where the coarse-score phase switches to 16-row items):
+    kept blocks and routing bit-exact, the stage intermediates and sampled output rows close."""
+    import torch
+    import block_sparse_attention_isa_b200 as isa
+    from parity_util import to_device
+    w = _case("many_blocks", 1, 2, 64, 20480, 20480, 64, 0.25, 0.5)
+    q, k, v = inputs(w)
+    tq, tk, tv = (to_device(x, w) for x in (q, k, v))
+    out, sel, route = isa.forward(tq, tk, tv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, debug=True)
+    pooled = isa.debug_pooled(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s)
+    isa.device_status()
+    out = out.float().cpu().numpy()
+    rng = np.random.default_rng(5)
+    for h in range(w.H):
+        r = O.isa_select_route_ref(q[0, h], k[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+        np.testing.assert_array_equal(sel[0, h].cpu().numpy(), r["sel"])
+        np.testing.assert_array_equal(route[0, h].cpu().numpy(), np.concatenate([r["exact"], r["taylor"]]))
+        np.testing.assert_allclose(pooled["colscore"][0, h].cpu().numpy(), r["colscore"], rtol=1e-4, atol=1e-7)
+        np.testing.assert_allclose(pooled["sharp"][0, h].cpu().numpy(), r["sharp"], rtol=1e-3, atol=1e-9)
+        rows = np.sort(rng.choice(w.N, size=192, replace=False))
+        ref = O.isa_rows_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, rows, sr=r)
+        compare_out(out[0, h, rows], ref)
