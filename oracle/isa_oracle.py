@@ -52,6 +52,15 @@ the design notes):
 * Each query block takes exactly one path, so write-back is a scatter into
   the original token order with no merge.
 * The Taylor path is computed literally, with the block-length weight b.
+* No-sparsity ratio alpha_ns (papernotes.org, "Key design 2" block mask M_ij
+  and "Key design 3" "alpha_ns controls the in-block non-sparse share";
+  paperlayer.ai summary section 2 "Pooling Attention": top-k entries of the
+  coarse map give the block mask; section 4 defaults alpha_ns = 0.0625). For
+  a Taylor query block i, the k_ns = ceil(alpha_ns * n_new - 1e-4) key blocks
+  of K_new with the largest coarse scores softmax_j(Qc_i . Kc_new_j / sqrt(D))
+  (ties by lower index) are computed exactly, all of their b keys, and every
+  other block of K_new through its pooled row with weight b, in one softmax.
+  alpha_ns = 0 is the plain Taylor path. Exact query blocks are unaffected.
 """
 from __future__ import annotations
 
@@ -79,6 +88,10 @@ __all__ = [
     "topk_margin",
     "route_margin",
     "executed_flops",
+    "no_sparse_block_count",
+    "no_sparse_blocks",
+    "taylor_mixed_rows",
+    "no_sparse_margin",
 ]
 
 F64 = np.float64
@@ -228,6 +241,66 @@ def taylor_rows(q_rows: np.ndarray, k_new: np.ndarray, v_new: np.ndarray, b: int
     return num / den
 
 
+def no_sparse_block_count(alpha_ns: float, n_new: int) -> int:
+    """k_ns = ceil(alpha_ns * n_new - 1e-4) from the float32 ratio, clamped to [0, n_new].
+
+    papernotes.org, "Key design 3": alpha_ns is the share of a Taylor query
+    block's key blocks that are not made sparse; the count is rounded up like
+    the kept context blocks.
+    """
+    a = _f32(alpha_ns)
+    if a <= 0.0:
+        return 0
+    return int(min(n_new, max(0, math.ceil(a * n_new - 1e-4))))
+
+
+def no_sparse_blocks(p_row: np.ndarray, k_ns: int) -> np.ndarray:
+    """The k_ns key blocks of K_new with the largest coarse scores in one row, ascending.
+
+    paperlayer.ai summary, section 2: top-k entries of the coarse attention map
+    give the block mask. Ranked by (score descending, index ascending).
+    """
+    order = sorted(range(len(p_row)), key=lambda j: (-float(p_row[j]), j))
+    return np.array(sorted(order[:k_ns]), dtype=np.int64)
+
+
+def taylor_mixed_rows(q_rows: np.ndarray, k_new: np.ndarray, v_new: np.ndarray, b: int,
+                      exact_blocks: Sequence[int]) -> np.ndarray:
+    """Taylor attention with some key blocks computed exactly, in one softmax.
+
+    papernotes.org, "Key design 2": for M_ij = 1, S_ij = q K_j^T / sqrt(D) and
+    P_ij = exp(S_ij) over the block's keys, l += rowsum(P_ij), O += P_ij V_j;
+    for M_ij = 0, S^c_ij = q Kc_j^T / sqrt(D), P^c_ij = exp(S^c_ij),
+    l += P^c_ij * L_K, O += P^c_ij Vc_j * L_K (L_K = b); finally O = O / l.
+    The maximum over all terms is subtracted before exp (the ratio is unchanged).
+    """
+    d = q_rows.shape[1]
+    n_new = k_new.shape[0] // b
+    ex = sorted(set(int(j) for j in exact_blocks))
+    pooled = [j for j in range(n_new) if j not in set(ex)]
+    q64 = np.asarray(q_rows, F64)
+    kc_new = pool_blocks(k_new, b)
+    vc_new = pool_blocks(v_new, b)
+    rows = np.concatenate([np.arange(j * b, (j + 1) * b) for j in ex]) if ex else np.zeros(0, np.int64)
+    se = (q64 @ np.asarray(k_new, F64)[rows].T) / math.sqrt(d)      # exact keys
+    sc = (q64 @ kc_new[pooled].T) / math.sqrt(d)                     # pooled blocks
+    m = np.maximum(se.max(axis=1, initial=-np.inf), sc.max(axis=1, initial=-np.inf))[:, None]
+    pe = np.exp(se - m)
+    pc = np.exp(sc - m) * b
+    num = pe @ np.asarray(v_new, F64)[rows] + pc @ vc_new[pooled]
+    den = pe.sum(axis=1, keepdims=True) + pc.sum(axis=1, keepdims=True)
+    return num / den
+
+
+def no_sparse_margin(p_rows: np.ndarray, k_ns: int) -> float:
+    """Smallest relative gap, over the given coarse rows, between their k_ns-th and (k_ns+1)-th scores."""
+    if k_ns <= 0 or p_rows.shape[1] <= k_ns or p_rows.shape[0] == 0:
+        return float("inf")
+    srt = -np.sort(-p_rows, axis=1)
+    a, c = srt[:, k_ns - 1], srt[:, k_ns]
+    return float(np.min((a - c) / np.maximum(np.abs(a), 1e-300)))
+
+
 def _validate(N: int, L_src: int, L_ctx: int, b: int):
     if L_src + L_ctx != N:
         raise ValueError("N must equal L_src + L_ctx")
@@ -236,12 +309,14 @@ def _validate(N: int, L_src: int, L_ctx: int, b: int):
 
 
 def isa_select_route_ref(q: np.ndarray, k: np.ndarray, L_src: int, L_ctx: int, b: int,
-                         alpha_s: float, alpha_f: float) -> Dict[str, np.ndarray]:
+                         alpha_s: float, alpha_f: float, alpha_ns: float = 0.0) -> Dict[str, np.ndarray]:
     """Stages 1-3 for one [N, D] slice: pooling probe, pre-selection, routing.
 
     Returns the pooled Qc/Kc, the coarse map's context scores, the kept blocks
     ``sel``, the sharpness M over all query blocks, the routing and the two
-    tie margins used to reject near-tie inputs.
+    tie margins used to reject near-tie inputs. With alpha_ns > 0 also the
+    exactly computed key blocks of every query block (``ns_sel``, [n_q, k_ns])
+    and the tie margin of that choice over the Taylor blocks.
     """
     N, D = q.shape
     _validate(N, L_src, L_ctx, b)
@@ -256,24 +331,33 @@ def isa_select_route_ref(q: np.ndarray, k: np.ndarray, L_src: int, L_ctx: int, b
     k_new_pooled = np.concatenate([kc[:n_src], kc[n_src + sel]], axis=0) if kk else kc[:n_src]
     m = sharpness(qc, k_new_pooled)
     exact, taylor = route_blocks(m, n_flat)
+    n_new = k_new_pooled.shape[0]
+    k_ns = no_sparse_block_count(alpha_ns, n_new)
+    p_new = coarse_scores(qc, k_new_pooled) if k_ns else np.zeros((n_q, n_new))
+    ns_sel = np.stack([no_sparse_blocks(p_new[i], k_ns) for i in range(n_q)]) if k_ns else np.zeros((n_q, 0), np.int64)
     return dict(qc=qc, kc=kc, s_coarse=s_coarse, colscore=colscore, sel=sel, kc_new=k_new_pooled,
-                sharp=m, exact=exact, taylor=taylor, k=kk, n_flat=n_flat,
-                topk_margin=topk_margin(colscore, kk), route_margin=route_margin(m, n_flat))
+                sharp=m, exact=exact, taylor=taylor, k=kk, n_flat=n_flat, k_ns=k_ns, ns_sel=ns_sel,
+                topk_margin=topk_margin(colscore, kk), route_margin=route_margin(m, n_flat),
+                ns_margin=no_sparse_margin(p_new[taylor], k_ns) if k_ns else float("inf"))
 
 
 def isa_slice_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, L_src: int, L_ctx: int, b: int,
-                  alpha_s: float, alpha_f: float, row_chunk: int = 2048) -> Dict[str, np.ndarray]:
+                  alpha_s: float, alpha_f: float, row_chunk: int = 2048, alpha_ns: float = 0.0) -> Dict[str, np.ndarray]:
     """The whole forward pass for one (batch, head) slice of [N, D] arrays.
 
     Rows are processed in chunks of ``row_chunk`` to bound memory; every row's
     softmax still runs over all of its keys in one piece.
     """
     N, D = q.shape
-    r = isa_select_route_ref(q, k, L_src, L_ctx, b, alpha_s, alpha_f)
+    r = isa_select_route_ref(q, k, L_src, L_ctx, b, alpha_s, alpha_f, alpha_ns)
     k_new, v_new = gather_kv(k, v, r["sel"], L_src, b)
     out = np.zeros((N, D), F64)
+    if r["k_ns"]:  # mixed Taylor path: each flat block with its own exactly computed key blocks
+        for i in r["taylor"]:
+            rr = np.arange(i * b, (i + 1) * b)
+            out[rr] = taylor_mixed_rows(q[rr], k_new, v_new, b, r["ns_sel"][i])
     for blocks, fn in ((r["exact"], "exact"), (r["taylor"], "taylor")):
-        if len(blocks) == 0:
+        if len(blocks) == 0 or (fn == "taylor" and r["k_ns"]):
             continue
         rows = np.concatenate([np.arange(i * b, (i + 1) * b) for i in blocks])
         for s in range(0, len(rows), row_chunk):
@@ -289,10 +373,10 @@ def isa_slice_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, L_src: int, L_ctx
 
 def isa_rows_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, L_src: int, L_ctx: int, b: int,
                  alpha_s: float, alpha_f: float, rows: Sequence[int],
-                 sr: Optional[Dict[str, np.ndarray]] = None) -> np.ndarray:
+                 sr: Optional[Dict[str, np.ndarray]] = None, alpha_ns: float = 0.0) -> np.ndarray:
     """Output rows ``rows`` of one slice only (for sampled checks at full size)."""
     if sr is None:
-        sr = isa_select_route_ref(q, k, L_src, L_ctx, b, alpha_s, alpha_f)
+        sr = isa_select_route_ref(q, k, L_src, L_ctx, b, alpha_s, alpha_f, alpha_ns)
     k_new, v_new = gather_kv(k, v, sr["sel"], L_src, b)
     taylor = set(int(t) for t in sr["taylor"])
     rows = np.asarray(rows, dtype=np.int64)
@@ -301,12 +385,17 @@ def isa_rows_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, L_src: int, L_ctx:
     if (~is_t).any():
         out[~is_t] = exact_rows(q[rows[~is_t]], k_new, v_new)
     if is_t.any():
-        out[is_t] = taylor_rows(q[rows[is_t]], k_new, v_new, b)
+        if sr.get("k_ns", 0):
+            for n, r_ in enumerate(rows):
+                if is_t[n]:
+                    out[n] = taylor_mixed_rows(q[[r_]], k_new, v_new, b, sr["ns_sel"][int(r_) // b])[0]
+        else:
+            out[is_t] = taylor_rows(q[rows[is_t]], k_new, v_new, b)
     return out
 
 
 def isa_forward_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, L_src: int, L_ctx: int, b: int,
-                    alpha_s: float, alpha_f: float) -> Dict[str, np.ndarray]:
+                    alpha_s: float, alpha_f: float, alpha_ns: float = 0.0) -> Dict[str, np.ndarray]:
     """Whole forward pass for [B, H, N, D] inputs; slices are independent.
 
     Returns ``out`` [B,H,N,D] (float64), ``sel`` [B,H,k] and ``route``
@@ -316,7 +405,7 @@ def isa_forward_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, L_src: int, L_c
     outs, sels, routes = [], [], []
     for bi in range(B):
         for h in range(H):
-            r = isa_slice_ref(q[bi, h], k[bi, h], v[bi, h], L_src, L_ctx, b, alpha_s, alpha_f)
+            r = isa_slice_ref(q[bi, h], k[bi, h], v[bi, h], L_src, L_ctx, b, alpha_s, alpha_f, alpha_ns=alpha_ns)
             outs.append(r["out"])
             sels.append(r["sel"])
             routes.append(r["route"])

@@ -342,3 +342,155 @@ def test_planted_mistakes(monkeypatch, name, fn):
     assert _pins_pass()
     monkeypatch.setattr(O, name, fn)
     assert not _pins_pass(), f"a planted mistake in {name} went unnoticed"
+
+
+# ----------------------------------------------------------------------------- no-sparsity ratio alpha_ns
+
+@pytest.mark.parametrize("a_ns,n_new,k", [(0.0, 160, 0), (0.0625, 160, 10), (0.0625, 16, 1), (0.0625, 24, 2),
+                                          (1.0, 37, 37), (0.1, 200, 20), (0.5, 5, 3)])
+def test_no_sparse_block_count(a_ns, n_new, k):
+    assert O.no_sparse_block_count(a_ns, n_new) == k
+
+
+def test_no_sparse_blocks_brute_force():
+    rng = np.random.default_rng(11)
+    for _ in range(200):
+        n = int(rng.integers(1, 12))
+        row = rng.integers(0, 4, size=n).astype(float) / 7.0  # many ties
+        for k_ns in range(n + 1):
+            ranked = sorted(((-row[j], j) for j in range(n)))
+            want = sorted(j for _, j in ranked[:k_ns])
+            assert O.no_sparse_blocks(row, k_ns).tolist() == want
+
+
+def _mixed_by_loops(q_rows, k_new, v_new, b, exact_blocks):
+    """The definition's sums written out with scalar loops: exact keys with weight 1, every
+    other block's pooled key and value with weight b, then the ratio."""
+    d = q_rows.shape[1]
+    n_new = k_new.shape[0] // b
+    out = np.zeros((q_rows.shape[0], d))
+    for r in range(q_rows.shape[0]):
+        terms = []  # (score, weight, value vector)
+        for j in range(n_new):
+            if j in exact_blocks:
+                for t in range(j * b, (j + 1) * b):
+                    s = sum(float(q_rows[r, x]) * float(k_new[t, x]) for x in range(d)) / math.sqrt(d)
+                    terms.append((s, 1.0, [float(v_new[t, x]) for x in range(d)]))
+            else:
+                kc = [sum(float(k_new[t, x]) for t in range(j * b, (j + 1) * b)) / b for x in range(d)]
+                vc = [sum(float(v_new[t, x]) for t in range(j * b, (j + 1) * b)) / b for x in range(d)]
+                s = sum(float(q_rows[r, x]) * kc[x] for x in range(d)) / math.sqrt(d)
+                terms.append((s, float(b), vc))
+        num = [0.0] * d
+        den = 0.0
+        for s, wgt, vec in terms:
+            e = wgt * math.exp(s)
+            den += e
+            for x in range(d):
+                num[x] += e * vec[x]
+        out[r] = [n / den for n in num]
+    return out
+
+
+def test_mixed_taylor_brute_force_loops():
+    rng = np.random.default_rng(3)
+    for b, n_new, D in [(2, 4, 3), (3, 5, 2), (4, 3, 4)]:
+        q = rng.standard_normal((5, D))
+        k = rng.standard_normal((n_new * b, D))
+        v = rng.standard_normal((n_new * b, D))
+        for ex in ([], [0], [1, 2], list(range(n_new))):
+            np.testing.assert_allclose(O.taylor_mixed_rows(q, k, v, b, ex), _mixed_by_loops(q, k, v, b, ex),
+                                       rtol=1e-12, atol=1e-13)
+
+
+def test_mixed_taylor_limits():
+    """No exact block: the plain Taylor path. Every block exact: exact attention over K_new."""
+    rng = np.random.default_rng(4)
+    b, n_new, D = 8, 6, 16
+    q = rng.standard_normal((10, D))
+    k = rng.standard_normal((n_new * b, D))
+    v = rng.standard_normal((n_new * b, D))
+    np.testing.assert_allclose(O.taylor_mixed_rows(q, k, v, b, []), O.taylor_rows(q, k, v, b), rtol=1e-12)
+    np.testing.assert_allclose(O.taylor_mixed_rows(q, k, v, b, range(n_new)), _sdpa(q, k, v), rtol=1e-11, atol=1e-13)
+
+
+def test_mixed_taylor_constant_keys_ignore_selection():
+    """Keys constant inside every block: an exact block contributes exp(s_j) * b * Vc_j, the same as
+    its pooled stand-in, so any choice of exact blocks gives dense attention."""
+    rng = np.random.default_rng(5)
+    b, n_new, D = 4, 7, 8
+    kc = rng.standard_normal((n_new, D))
+    k = np.repeat(kc, b, axis=0)
+    v = rng.standard_normal((n_new * b, D))
+    q = rng.standard_normal((6, D))
+    dense = _sdpa(q, k, v)
+    for ex in ([], [3], [0, 6], [1, 2, 4, 5]):
+        np.testing.assert_allclose(O.taylor_mixed_rows(q, k, v, b, ex), dense, rtol=1e-11, atol=1e-13)
+
+
+def test_mixed_taylor_split_and_merge():
+    """One softmax over the two key sets equals the merge of the two partial softmaxes
+    (running max, sum and unnormalised output), the identity an online softmax relies on."""
+    rng = np.random.default_rng(6)
+    b, n_new, D = 4, 6, 8
+    q = rng.standard_normal((5, D))
+    k = rng.standard_normal((n_new * b, D))
+    v = rng.standard_normal((n_new * b, D))
+    ex = [1, 4]
+    rows = np.concatenate([np.arange(j * b, (j + 1) * b) for j in ex])
+    pooled = [j for j in range(n_new) if j not in ex]
+    kc, vc = O.pool_blocks(k, b)[pooled], O.pool_blocks(v, b)[pooled]
+    s1 = q @ k[rows].T / math.sqrt(D)
+    s2 = q @ kc.T / math.sqrt(D) + math.log(b)  # weight b as a score bias
+    parts = []
+    for s, vv in ((s1, v[rows]), (s2, vc)):
+        m = s.max(1, keepdims=True)
+        p = np.exp(s - m)
+        parts.append((m, p.sum(1, keepdims=True), p @ vv))
+    m = np.maximum(parts[0][0], parts[1][0])
+    l = sum(li * np.exp(mi - m) for mi, li, _ in parts)
+    o = sum(oi * np.exp(mi - m) for mi, _, oi in parts)
+    np.testing.assert_allclose(o / l, O.taylor_mixed_rows(q, k, v, b, ex), rtol=1e-12)
+
+
+def test_slice_with_no_sparse_blocks():
+    """A whole slice at alpha_ns = 0 is unchanged; at alpha_ns > 0 only the Taylor rows change, each
+    flat block using its own top coarse-score key blocks."""
+    w = _small(D=16, b=8, L_src=64, L_ctx=64, a_s=0.5, a_f=0.5)
+    q, k, v = isa_synth.make_slice(w, 0, 0, 0)
+    base = O.isa_slice_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+    same = O.isa_slice_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, alpha_ns=0.0)
+    np.testing.assert_array_equal(base["out"], same["out"])
+    ns = O.isa_slice_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, alpha_ns=0.25)
+    n_new = ns["kc_new"].shape[0]
+    assert ns["k_ns"] == math.ceil(0.25 * n_new) and ns["ns_sel"].shape == (16, ns["k_ns"])
+    p = O.coarse_scores(ns["qc"], ns["kc_new"])
+    k_new, v_new = O.gather_kv(k, v, ns["sel"], w.L_src, w.b)
+    for i in range(16):
+        rr = slice(i * w.b, (i + 1) * w.b)
+        if i in set(ns["exact"].tolist()):
+            np.testing.assert_array_equal(ns["out"][rr], base["out"][rr])
+        else:
+            want = set(np.argsort(-p[i], kind="stable")[:ns["k_ns"]].tolist())
+            assert set(ns["ns_sel"][i].tolist()) == want
+            np.testing.assert_allclose(ns["out"][rr], _mixed_by_loops(q[rr], k_new, v_new, w.b, want), rtol=1e-10)
+
+
+def _mixed_wrong(q_rows, k_new, v_new, b, exact_blocks):
+    """A plausible slip: the pooled blocks lose their weight b."""
+    d = q_rows.shape[1]
+    n_new = k_new.shape[0] // b
+    ex = sorted(set(int(j) for j in exact_blocks))
+    pooled = [j for j in range(n_new) if j not in ex]
+    kc, vc = O.pool_blocks(k_new, b)[pooled], O.pool_blocks(v_new, b)[pooled]
+    rows = np.concatenate([np.arange(j * b, (j + 1) * b) for j in ex]) if ex else np.zeros(0, np.int64)
+    s = np.concatenate([q_rows @ k_new[rows].T, q_rows @ kc.T], axis=1) / math.sqrt(d)
+    p = np.exp(s - s.max(1, keepdims=True))
+    vv = np.concatenate([v_new[rows], vc], axis=0)
+    return (p @ vv) / p.sum(1, keepdims=True)
+
+
+def test_planted_mistake_in_mixed_path(monkeypatch):
+    monkeypatch.setattr(O, "taylor_mixed_rows", _mixed_wrong)
+    with pytest.raises(AssertionError):
+        test_mixed_taylor_brute_force_loops()
