@@ -40,17 +40,28 @@ BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 # ----------------------------------------------------------------------------- host-side logic (tested on CPU)
 
-def flops_per_call(w) -> dict:
-    """Multiply-adds of each stage x 2 for one call over all B*H slices (the pass's own counts)."""
+def no_sparse_count(alpha_ns: float, n_new: int) -> int:
+    """k_ns = ceil(alpha_ns * n_new - 1e-4) exact key blocks per Taylor query block (0 for alpha_ns = 0)."""
+    if alpha_ns <= 0:
+        return 0
+    return max(0, min(n_new, math.ceil(float(np.float32(alpha_ns)) * n_new - 1e-4)))
+
+
+def flops_per_call(w, alpha_ns: float = 0.0) -> dict:
+    """Multiply-adds of each stage x 2 for one call over all B*H slices (the pass's own counts).
+
+    With alpha_ns > 0 a Taylor query row attends to the n_new - k_ns pooled rows
+    and the k_ns * b keys of its exact blocks."""
     N = w.L_src + w.L_ctx
     n_q, n_src, n_ctx = N // w.b, w.L_src // w.b, w.L_ctx // w.b
     k = max(0, min(n_ctx, math.ceil(float(np.float32(w.alpha_s)) * n_ctx - 1e-4)))
     n_flat = max(0, min(n_q, math.floor(float(np.float32(w.alpha_f)) * n_q + 1e-4)))
     n_new = n_src + k
+    k_ns = no_sparse_count(alpha_ns, n_new)
     bh = w.B * w.H
     f = dict(coarse=2.0 * n_src * n_q * w.D * bh, route=2.0 * n_q * n_new * w.D * bh,
              exact=4.0 * (n_q - n_flat) * w.b * n_new * w.b * w.D * bh,
-             taylor=4.0 * n_flat * w.b * n_new * w.D * bh)
+             taylor=4.0 * n_flat * w.b * ((n_new - k_ns) + k_ns * w.b) * w.D * bh)
     f["total"] = sum(f.values())
     return f
 
@@ -163,19 +174,24 @@ def bf16_bits(x):
     return isa_synth.round_to_bf16_bits(x)
 
 
-def cpu_oracle_sample(w, q, k, v, heads, seconds_cap=60.0):
+def cpu_oracle_sample(w, q, k, v, heads, seconds_cap=60.0, alpha_ns=0.0):
     """Run the oracle on some heads; returns (TFLOP/s, seconds, heads done)."""
     from oracle import isa_oracle as O
-    f = flops_per_call(w)["total"] / (w.B * w.H)
+    f = flops_per_call(w, alpha_ns)["total"] / (w.B * w.H)
     t0 = time.perf_counter()
     done = 0
     for h in heads:
-        O.isa_slice_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+        O.isa_slice_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, alpha_ns=alpha_ns)
         done += 1
         if time.perf_counter() - t0 > seconds_cap:
             break
     dt = time.perf_counter() - t0
     return f * done / dt / 1e12, dt, done
+
+
+def workload_label(args, w) -> str:
+    label = w.name + (f" (first {w.H} heads)" if args.heads else "")
+    return label + (f", alpha_ns={args.alpha_ns:g}" if args.alpha_ns else "")
 
 
 def run_reference(args, w):
@@ -198,16 +214,20 @@ def run_reference(args, w):
     n_new = w.L_src // w.b + kk
     per_head = O.executed_flops(1, 1, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, w.alpha_f)
     sel_route_flops = per_head["coarse"] + per_head["route"]
+    a_ns = args.alpha_ns
+    k_ns = no_sparse_count(a_ns, n_new)
 
     def step(s):
         h = s % n_heads
-        sr = O.isa_select_route_ref(q[0, h], k[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+        sr = O.isa_select_route_ref(q[0, h], k[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, a_ns)
         blocks = np.arange(s % parts, n_q, parts)
         rows = (blocks[:, None] * w.b + np.arange(w.b)[None, :]).ravel()
-        O.isa_rows_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, rows, sr=sr)
+        O.isa_rows_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, rows, sr=sr,
+                       alpha_ns=a_ns)
         taylor = set(int(t) for t in sr["taylor"])
         n_t = sum(int(bl) in taylor for bl in blocks)
-        return sel_route_flops + 4.0 * w.b * w.D * ((len(blocks) - n_t) * n_new * w.b + n_t * n_new)
+        return sel_route_flops + 4.0 * w.b * w.D * ((len(blocks) - n_t) * n_new * w.b +
+                                                     n_t * ((n_new - k_ns) + k_ns * w.b))
 
     for s in range(args.warmup):
         step(s)
@@ -222,8 +242,9 @@ def run_reference(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": w.name + (f" (first {w.H} heads)" if args.heads else ""), "B": w.B, "H": w.H,
-                       "N": w.N, "D": w.D, "b": w.b, "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "sample": sample},
+            "config": {"workload": workload_label(args, w), "B": w.B, "H": w.H,
+                       "N": w.N, "D": w.D, "b": w.b, "alpha_s": w.alpha_s, "alpha_f": w.alpha_f,
+                       "alpha_ns": args.alpha_ns, "sample": sample},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -250,13 +271,15 @@ def run_ours(args, w):
     q, k, v = workload_inputs(w, full=getattr(args, "full_workload", None))
     tq, tk, tv = (torch.from_numpy(x).to(dev, dt) for x in (q, k, v))
     out = torch.empty_like(tq)
+    a_ns = args.alpha_ns
     ws = torch.empty(isa.workspace_bytes(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s,
-                                         isa.ISA_BF16 if w.dtype == "bf16" else isa.ISA_F32),
+                                         isa.ISA_BF16 if w.dtype == "bf16" else isa.ISA_F32, alpha_ns=a_ns),
                      dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        isa.forward_into(tq, tk, tv, out, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, workspace=ws, stream=stream)
+        isa.forward_into(tq, tk, tv, out, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, workspace=ws, stream=stream,
+                         alpha_ns=a_ns)
 
     for _ in range(args.warmup):
         step()
@@ -292,7 +315,7 @@ def run_ours(args, w):
     max_ms = reduce_max(ms, dist)
     stage_ms = {name: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)) / args.steps
                 for i, name in enumerate(isa.STAGES)}
-    f = flops_per_call(w)
+    f = flops_per_call(w, a_ns)
     hb = hbm_bytes_per_call(w)
     peaks, peaks_kind = load_peaks()
     attn_tflops = (f["exact"] + f["taylor"]) / (stage_ms["attention"] * 1e-3) / 1e12
@@ -301,7 +324,7 @@ def run_ours(args, w):
     gather_gbs = hb["gather"] / max(stage_ms["gather"] * 1e-3, 1e-12) / 1e9
     traffic = None
     prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof):
+    if os.path.exists(prof) and not a_ns:  # (the counters cover the plain path's attention kernel only)
         with open(prof) as fh:
             ent = json.load(fh).get(w.name, {})
         # the counters hold only for the kernel source they were taken on
@@ -310,7 +333,8 @@ def run_ours(args, w):
 
     # end to end through the host-buffer entry point (pinned host memory, copies inside the timed region)
     e2e = None
-    if not args.no_e2e and (rank == 0 or world > 1):
+    # (the host-buffer entry point has no alpha_ns argument: no end-to-end figure for that variant)
+    if not args.no_e2e and not a_ns and (rank == 0 or world > 1):
         hq, hk, hv = (t.cpu().pin_memory() for t in (tq, tk, tv))
         hout = torch.empty_like(hq).pin_memory()
         n_e2e = max(1, min(args.steps, 5))
@@ -327,20 +351,21 @@ def run_ours(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, secs, done = cpu_oracle_sample(w, q, k, v, heads=range(w.H), seconds_cap=args.cpu_seconds)
+        tf, secs, done = cpu_oracle_sample(w, q, k, v, heads=range(w.H), seconds_cap=args.cpu_seconds,
+                                           alpha_ns=a_ns)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
                "sample": f"{done} of {w.B * w.H} heads of the same workload, {secs:.1f} s of CPU time"}
 
     launches = isa.launch_count(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, w.alpha_f,
-                                isa.ISA_BF16 if w.dtype == "bf16" else isa.ISA_F32)
+                                isa.ISA_BF16 if w.dtype == "bf16" else isa.ISA_F32, alpha_ns=a_ns)
     if rank == 0:
         line = {
             "metric": METRIC, "value": aggregate(f["total"], max_ms, world), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
             "data": "synthetic",
-            "config": {"workload": w.name + (f" (first {w.H} heads)" if args.heads else ""), "B": w.B, "H": w.H, "N": w.N, "D": w.D, "b": w.b,
-                       "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "global_batch": w.B * world,
+            "config": {"workload": workload_label(args, w), "B": w.B, "H": w.H, "N": w.N, "D": w.D, "b": w.b,
+                       "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "alpha_ns": a_ns, "global_batch": w.B * world,
                        "seq_len": w.N, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (Q, K, V = %.2f GB per step)" % (3 * tq.numel() * tq.element_size() / 1e9)},
             "roofline": {"bound": "tensor", "kernel": "attention (exact + Taylor paths)", "achieved": attn_tflops,
@@ -373,6 +398,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--alpha-ns", type=float, default=0.0,
+                    help="no-sparsity ratio: exact key blocks inside the Taylor path (bf16 only; 0 = plain path)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run only the first H heads of the workload (small profiling captures; not a bench line)")
     args = ap.parse_args()

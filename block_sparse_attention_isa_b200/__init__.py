@@ -19,6 +19,7 @@ __all__ = [
     "lib",
     "lib_path",
     "plan",
+    "plan_ns",
     "workspace_bytes",
     "launch_count",
     "forward",
@@ -60,6 +61,10 @@ EXPORTS = (
     "isa_selftest_exp2",
     "isa_set_stage_events",
     "isa_select_context_noalloc",
+    "isa_plan_ns",
+    "isa_workspace_bytes_ns",
+    "isa_forward_ns",
+    "isa_launch_count_ns",
     "isa_last_error",
 )
 
@@ -115,6 +120,15 @@ def lib() -> ctypes.CDLL:
     L.isa_set_stage_events.restype = c_int
     L.isa_select_context_noalloc.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_int, vp, vp, vp]
     L.isa_select_context_noalloc.restype = c_int
+    L.isa_plan_ns.argtypes = [c_int] * 6 + [c_float, c_float, c_float, i32p, i32p, i32p, i32p]
+    L.isa_plan_ns.restype = c_int
+    L.isa_workspace_bytes_ns.argtypes = [c_int] * 6 + [c_float, c_float, c_int]
+    L.isa_workspace_bytes_ns.restype = c_size
+    L.isa_forward_ns.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_float, c_float, c_int, vp, vp, vp, vp, vp,
+                                                              c_size, vp]
+    L.isa_forward_ns.restype = c_int
+    L.isa_launch_count_ns.argtypes = [c_int] * 6 + [c_float, c_float, c_float, c_int]
+    L.isa_launch_count_ns.restype = c_int
     L.isa_last_error.argtypes = []
     L.isa_last_error.restype = ctypes.c_char_p
     _LIB = L
@@ -138,14 +152,27 @@ def plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f) -> Tuple[int, int, int]:
     return n_q.value, k.value, n_flat.value
 
 
-def workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dtype=ISA_BF16) -> int:
-    n = lib().isa_workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dtype)
+def plan_ns(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, alpha_ns) -> Tuple[int, int, int, int]:
+    """(n_q, k, n_flat, k_ns): plan() plus the exact key blocks per Taylor query block."""
+    n_q, k, n_flat, k_ns = (ctypes.c_int32() for _ in range(4))
+    _check(lib().isa_plan_ns(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, alpha_ns, ctypes.byref(n_q),
+                             ctypes.byref(k), ctypes.byref(n_flat), ctypes.byref(k_ns)))
+    return n_q.value, k.value, n_flat.value, k_ns.value
+
+
+def workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dtype=ISA_BF16, alpha_ns: float = 0.0) -> int:
+    if alpha_ns:
+        n = lib().isa_workspace_bytes_ns(B, H, L_src, L_ctx, D, b, alpha_s, alpha_ns, dtype)
+    else:
+        n = lib().isa_workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dtype)
     if n == 0:
         raise IsaError(-1, last_error())
     return n
 
 
-def launch_count(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dtype=ISA_BF16) -> int:
+def launch_count(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dtype=ISA_BF16, alpha_ns: float = 0.0) -> int:
+    if alpha_ns:
+        return lib().isa_launch_count_ns(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, alpha_ns, dtype)
     return lib().isa_launch_count(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dtype)
 
 
@@ -177,12 +204,15 @@ def _workspace(device, nbytes: int):
 
 
 def forward_into(q, k, v, out, L_src: int, L_ctx: int, b: int, alpha_s: float, alpha_f: float,
-                 dbg_sel=None, dbg_route=None, workspace=None, stream=None):
+                 dbg_sel=None, dbg_route=None, workspace=None, stream=None, alpha_ns: float = 0.0, dbg_ns=None):
     """Enqueue the pass on ``stream`` (default: torch's current stream) writing ``out``.
 
     All tensors are CUDA tensors; q, k, v, out are contiguous [B, H, N, D] of one
     dtype (bfloat16 or float32); dbg_sel int32 [B, H, k] and dbg_route int32
-    [B, H, n_q] are optional. Asynchronous; returns the workspace used.
+    [B, H, n_q] are optional. With ``alpha_ns`` > 0 (bfloat16 only) the Taylor
+    query blocks compute their k_ns best K_new blocks exactly (isa_forward_ns);
+    dbg_ns int32 [B, H, n_q, k_ns] then receives those blocks. Asynchronous;
+    returns the workspace used.
     """
     torch = _torch()
     for t in (q, k, v, out):
@@ -191,10 +221,17 @@ def forward_into(q, k, v, out, L_src: int, L_ctx: int, b: int, alpha_s: float, a
     B, H, N, D = q.shape
     dt = _dtype_code(q)
     if workspace is None:
-        workspace = _workspace(q.device, workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dt))
+        workspace = _workspace(q.device, workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dt, alpha_ns))
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     s = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    if alpha_ns or dbg_ns is not None:
+        _check(lib().isa_forward_ns(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, alpha_ns, dt,
+            out.data_ptr(), dbg_sel.data_ptr() if dbg_sel is not None else None,
+            dbg_route.data_ptr() if dbg_route is not None else None,
+            dbg_ns.data_ptr() if dbg_ns is not None else None, workspace.data_ptr(), workspace.numel(), s))
+        return workspace
     rc = lib().isa_forward_ex(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dt, out.data_ptr(),
         dbg_sel.data_ptr() if dbg_sel is not None else None, dbg_route.data_ptr() if dbg_route is not None else None,
@@ -204,18 +241,24 @@ def forward_into(q, k, v, out, L_src: int, L_ctx: int, b: int, alpha_s: float, a
 
 
 def forward(q, k, v, L_src: int, L_ctx: int, b: int, alpha_s: float, alpha_f: float, debug: bool = False,
-            stream=None):
-    """ISA forward pass on CUDA tensors; returns out, or (out, sel, route) when ``debug``."""
+            stream=None, alpha_ns: float = 0.0):
+    """ISA forward pass on CUDA tensors; returns out, or (out, sel, route) when ``debug``
+    ((out, sel, route, ns) with ``alpha_ns`` > 0, ns int32 [B, H, n_q, k_ns])."""
     torch = _torch()
     out = torch.empty_like(q)
-    sel = route = None
+    sel = route = ns = None
     if debug:
         B, H, N, D = q.shape
-        n_q, kk, _ = plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f)
+        n_q, kk, _, k_ns = plan_ns(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, alpha_ns)
         sel = torch.empty((B, H, kk), dtype=torch.int32, device=q.device)
         route = torch.empty((B, H, n_q), dtype=torch.int32, device=q.device)
-    forward_into(q, k, v, out, L_src, L_ctx, b, alpha_s, alpha_f, sel, route, stream=stream)
-    return (out, sel, route) if debug else out
+        if alpha_ns:
+            ns = torch.empty((B, H, n_q, k_ns), dtype=torch.int32, device=q.device)
+    forward_into(q, k, v, out, L_src, L_ctx, b, alpha_s, alpha_f, sel, route, stream=stream, alpha_ns=alpha_ns,
+                 dbg_ns=ns)
+    if not debug:
+        return out
+    return (out, sel, route, ns) if alpha_ns else (out, sel, route)
 
 
 def device_status(workspace=None, stream=None):

@@ -48,11 +48,19 @@ int flat_blocks(float alpha_f, int n_q) {
 
 bool ratio_ok(float a) { return !std::isnan(a) && a >= 0.0f && a <= 1.0f; }
 
-int make_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, int dt, Plan* p) {
+// Exactly computed key blocks per Taylor query block: ceil(alpha_ns * n_new) with a 1e-4 guard.
+int no_sparse_blocks(float alpha_ns, int n_new) {
+  if (!(alpha_ns > 0.0f)) return 0;
+  return kept_blocks(alpha_ns, n_new);
+}
+
+int make_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, int dt, Plan* p,
+              float alpha_ns = 0.0f) {
   if (B <= 0 || H <= 0) return fail(ISA_ERR_ARG, "B and H must be positive (B=%d H=%d)", B, H);
   if (L_src <= 0 || L_ctx <= 0) return fail(ISA_ERR_ARG, "L_src and L_ctx must be positive (%d, %d)", L_src, L_ctx);
   if (!ratio_ok(alpha_s) || !ratio_ok(alpha_f))
     return fail(ISA_ERR_ARG, "alpha_s and alpha_f must lie in [0, 1] (%g, %g)", (double)alpha_s, (double)alpha_f);
+  if (!ratio_ok(alpha_ns)) return fail(ISA_ERR_ARG, "alpha_ns must lie in [0, 1] (%g)", (double)alpha_ns);
   if (dt != ISA_BF16 && dt != ISA_F32) return fail(ISA_ERR_UNSUPPORTED, "unknown dtype %d", dt);
   if (D != 64 && D != 128) return fail(ISA_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
   if (b != 64 && b != 128) return fail(ISA_ERR_UNSUPPORTED, "block size b must be 64 or 128 (got %d)", b);
@@ -83,6 +91,10 @@ int make_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, f
   p->n_exact = n_q - p->n_flat;
   p->dt = dt;
   p->elem = dt == ISA_BF16 ? 2 : 4;
+  p->k_ns = no_sparse_blocks(alpha_ns, p->n_new);
+  p->ns_words = (p->n_new + 31) / 32;
+  if (p->k_ns > 0 && dt != ISA_BF16)
+    return fail(ISA_ERR_UNSUPPORTED, "alpha_ns > 0 needs bfloat16 inputs");
   return ISA_OK;
 }
 
@@ -94,8 +106,9 @@ bool overlaps(const void* a, const void* b, size_t bytes) {
 
 }  // namespace
 
-int build_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, int dt, Plan* p) {
-  return make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dt, p);
+int build_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, int dt, Plan* p,
+               float alpha_ns) {
+  return make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dt, p, alpha_ns);
 }
 
 int set_error(int code, const char* fmt, ...) {
@@ -135,6 +148,10 @@ size_t workspace_layout(const Plan& p, Work* w, char* base) {
   if (p.dt == ISA_F32) {
     t.vtn = reinterpret_cast<float*>(take(sizeof(float) * BH * p.D * p.L_new));
     t.vct = reinterpret_cast<float*>(take(sizeof(float) * BH * p.D * vct_ld(p)));
+  }
+  if (p.k_ns > 0) {
+    t.nsel = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * BH * p.n_q * p.k_ns));
+    t.nsmask = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * BH * p.n_q * p.ns_words));
   }
   if (w) *w = t;
   return off;
@@ -183,9 +200,17 @@ int run_forward(const void* q, const void* k, const void* v, const Plan& p, void
   if ((e = launch_route(p, w, s)) != cudaSuccess) return cuda_fail(e, "routing launch");
   if ((e = launch_transpose_v(v, p, w, s)) != cudaSuccess) return cuda_fail(e, "V transpose launch");
   if ((e = mark(3, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
-  e = attention_pair_supported(p) ? launch_attention_pair(q, k, v, out, p, w, s, nullptr)
-                                  : launch_attention(q, k, v, out, p, w, s, nullptr);
-  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  {
+    // with alpha_ns > 0 the Taylor query blocks go to their own launch; the first one then
+    // takes the exact items only (its plan has no flat blocks; the route lists are unchanged)
+    Plan pe = p;
+    if (p.k_ns > 0) pe.n_flat = 0;
+    e = attention_pair_supported(pe) ? launch_attention_pair(q, k, v, out, pe, w, s, nullptr)
+                                     : launch_attention(q, k, v, out, pe, w, s, nullptr);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    if (p.k_ns > 0 && p.n_flat > 0 && (e = launch_attention_ns(q, k, v, out, p, w, s)) != cudaSuccess)
+      return cuda_fail(e, "mixed Taylor attention launch");
+  }
   if ((e = mark(4, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
   if (dbg_sel && p.k > 0) {
     e = cudaMemcpyAsync(dbg_sel, w.sel, sizeof(int32_t) * (size_t)p.BH * p.k, cudaMemcpyDeviceToDevice, s);
@@ -249,6 +274,49 @@ int isa_launch_count(int B, int H, int L_src, int L_ctx, int D, int b, float alp
   Plan p;
   if (make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p) != ISA_OK) return 0;
   return 3 + (p.k > 0 ? 1 : 0) + (p.dt == ISA_F32 ? 1 : 0);
+}
+
+int isa_plan_ns(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, float alpha_ns,
+                int32_t* n_q, int32_t* k, int32_t* n_flat, int32_t* k_ns) {
+  Plan p;
+  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, ISA_BF16, &p, alpha_ns);
+  if (rc != ISA_OK) return rc;
+  if (n_q) *n_q = p.n_q;
+  if (k) *k = p.k;
+  if (n_flat) *n_flat = p.n_flat;
+  if (k_ns) *k_ns = p.k_ns;
+  return ISA_OK;
+}
+
+size_t isa_workspace_bytes_ns(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_ns,
+                              isa_dtype dt) {
+  Plan p;
+  if (make_plan(B, H, L_src, L_ctx, D, b, alpha_s, 0.0f, (int)dt, &p, alpha_ns) != ISA_OK) return 0;
+  return workspace_layout(p, nullptr, nullptr);
+}
+
+int isa_launch_count_ns(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f,
+                        float alpha_ns, isa_dtype dt) {
+  Plan p;
+  if (make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p, alpha_ns) != ISA_OK) return 0;
+  return 3 + (p.k > 0 ? 1 : 0) + (p.dt == ISA_F32 ? 1 : 0) + (p.k_ns > 0 && p.n_flat > 0 ? 1 : 0);
+}
+
+int isa_forward_ns(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
+                   float alpha_s, float alpha_f, float alpha_ns, isa_dtype dt, void* out, int32_t* dbg_sel,
+                   int32_t* dbg_route, int32_t* dbg_ns, void* workspace, size_t workspace_bytes, void* stream) {
+  Plan p;
+  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p, alpha_ns);
+  if (rc != ISA_OK) return rc;
+  if ((rc = check_io(q, k, v, out, p)) != ISA_OK) return rc;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rc = run_forward(q, k, v, p, out, dbg_sel, dbg_route, workspace, workspace_bytes, s);
+  if (rc != ISA_OK || !dbg_ns || p.k_ns == 0) return rc;
+  Work w;
+  workspace_layout(p, &w, static_cast<char*>(workspace));
+  const cudaError_t e = cudaMemcpyAsync(dbg_ns, w.nsel, sizeof(int32_t) * (size_t)p.BH * p.n_q * p.k_ns,
+                                        cudaMemcpyDeviceToDevice, s);
+  return e == cudaSuccess ? ISA_OK : cuda_fail(e, "copying dbg_ns");
 }
 
 int isa_forward_ex(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,

@@ -20,6 +20,8 @@ struct Plan {
   int n_exact; // n_q - n_flat query blocks on the exact path
   int dt;      // 0 = bf16, 1 = fp32
   int elem;    // bytes per element
+  int k_ns;    // key blocks of K_new computed exactly inside each Taylor query block (0: plain Taylor path)
+  int ns_words;  // 32-bit words of one query block's exact-key-block bitmask (ceil(n_new / 32))
 };
 
 // Row length of the transposed pooled V rows (fp32 inputs): n_new rounded up to 4
@@ -45,6 +47,8 @@ struct Work {
   void* vsel;            // [BH, k*b, D]
   float* vtn;            // fp32 inputs only: [BH, D, L_new] V_new transposed
   float* vct;            // fp32 inputs only: [BH, D, vct_ld] pooled V_new rows transposed
+  int32_t* nsel;         // k_ns > 0 only: [BH, n_q, k_ns] exactly computed K_new blocks of each query block, ascending
+  uint32_t* nsmask;      // k_ns > 0 only: [BH, n_q, ns_words] the same blocks as a bitmask over K_new's blocks
 };
 
 constexpr int kCtrlWords = 64;
@@ -71,7 +75,8 @@ size_t workspace_layout(const Plan& p, Work* w, char* base);
 
 // Argument checks and block counts shared by the entry points (same rules and
 // messages as isa_forward_ex); returns ISA_OK or an error code.
-int build_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, int dt, Plan* p);
+int build_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, int dt, Plan* p,
+               float alpha_ns = 0.0f);
 // Sets the thread-local message returned by isa_last_error() and returns `code`.
 int set_error(int code, const char* fmt, ...);
 
@@ -86,6 +91,11 @@ cudaError_t launch_attention(const void* q, const void* k, const void* v, void* 
 bool attention_pair_supported(const Plan& p);
 cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, void* out, const Plan& p,
                                   const Work& w, cudaStream_t s, int* n_ctas);
+// Taylor query blocks with exactly computed key blocks (k_ns > 0, bf16): one query block per
+// work item, keys = the pooled K_new rows (weight b, the block's exact blocks masked) followed
+// by the keys of its exact blocks, in one online softmax.
+cudaError_t launch_attention_ns(const void* q, const void* k, const void* v, void* out, const Plan& p,
+                                const Work& w, cudaStream_t s);
 
 // One thread waits on an mbarrier that nothing arrives on; the bounded wait gives
 // up after `timeout_ms` and sets kErrSelftest in err[0].

@@ -35,6 +35,15 @@
 //  * lazy rescaling: the running max only moves when it grows by more than
 //    2^8, and only then is the O row rescaled in TMEM by its own thread;
 //  * exact items come first in the static schedule and Taylor items after.
+//
+// The same kernel, instantiated with NS = true, computes Taylor query blocks
+// with some key blocks kept exact (the no-sparsity ratio alpha_ns of
+// papernotes.org, Key design 3; Key design 2 gives the two kinds of terms and
+// their one softmax). Each query block u has its own set E_u of k_ns blocks of
+// K_new. An item (the Taylor blocks of two query tiles) walks first the pooled
+// rows of K_new, each weighted by b (a log2(b) bias on its exponent) and masked
+// for the row's own E_u, then the key tiles of the union of its blocks' E_u,
+// where every row masks the blocks outside its own E_u.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 #include <float.h>
@@ -88,6 +97,10 @@ struct AttnParams {
   const int32_t* route;
   void* out;
   uint32_t* err;
+  const uint32_t* nsmask;  // NS: [BH, n_q, ns_words] exact key blocks of every query block
+  int ns_words;            // NS: ceil(n_new / 32)
+  int npt;                 // NS: K/V tiles of the pooled rows, ceil(n_new / 128)
+  float bias_log2;         // NS: log2(b), the weight of a pooled row in the exponent
   int BH, N, b, L_src, n_q, n_exact, n_flat, L_new, n_new;
   int bpt;       // blocks per 128-row tile (128 / b)
   int bpi;       // blocks per item (2 tiles)
@@ -141,10 +154,34 @@ struct Cfg {
 
 struct Item {
   int bh, kind, nblk, ntiles, nkv, last_valid;
+  int nu;  // NS: blocks in the union of the item's exact key blocks
   int blk0, blk1, blk2, blk3;  // query blocks of the item (repeats of blk0 past nblk)
   __device__ __forceinline__ int blk(int u) const { return u == 0 ? blk0 : u == 1 ? blk1 : u == 2 ? blk2 : blk3; }
 };
 
+// NS: word `wd` of the union of the exact-block bitmasks of the item's query blocks
+__device__ __forceinline__ uint32_t union_word(const AttnParams& p, const Item& it, int wd) {
+  const uint32_t* m = p.nsmask + (size_t)it.bh * p.n_q * p.ns_words + wd;
+  uint32_t x = 0;
+  for (int u = 0; u < it.nblk; ++u) x |= __ldg(m + (size_t)it.blk(u) * p.ns_words);
+  return x;
+}
+
+// NS: walks the union of an item's exact key blocks in ascending order. Callers ask
+// for at most it.nu blocks; past the end it returns block 0.
+struct BlockCursor {
+  int wd = -1;
+  uint32_t bits = 0;
+  __device__ __forceinline__ int next(const AttnParams& p, const Item& it) {
+    while (bits == 0 && wd + 1 < p.ns_words) bits = union_word(p, it, ++wd);
+    if (bits == 0) return 0;
+    const int j = __ffs(bits) - 1;
+    bits &= bits - 1;
+    return 32 * wd + j;
+  }
+};
+
+template <bool NS>
 __device__ __forceinline__ Item decode_item(const AttnParams& p, int g) {
   Item it;
   int count, base, pp;
@@ -170,9 +207,19 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p, int g) {
   it.blk2 = it.nblk > 2 ? __ldg(lst + first + 2) : it.blk0;
   it.blk3 = it.nblk > 3 ? __ldg(lst + first + 3) : it.blk0;
   it.ntiles = (it.nblk + p.bpt - 1) / p.bpt;
-  const int rows = it.kind == 0 ? p.L_new : p.n_new;
-  it.nkv = (rows + kBN - 1) / kBN;
-  it.last_valid = rows - kBN * (it.nkv - 1);
+  if constexpr (NS) {
+    // pooled rows, then the union of the exact blocks, 128 / b blocks per K/V tile
+    int nu = 0;
+    for (int wd = 0; wd < p.ns_words; ++wd) nu += __popc(union_word(p, it, wd));
+    it.nu = nu;
+    it.nkv = p.npt + (nu + p.bpt - 1) / p.bpt;
+    it.last_valid = p.n_new - kBN * (p.npt - 1);  // of the last pooled tile
+  } else {
+    const int rows = it.kind == 0 ? p.L_new : p.n_new;
+    it.nu = 0;
+    it.nkv = (rows + kBN - 1) / kBN;
+    it.last_valid = rows - kBN * (it.nkv - 1);
+  }
   return it;
 }
 
@@ -217,13 +264,14 @@ __device__ __forceinline__ void store_row_chunk<float>(float* dst, const float* 
   for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
 
-template <typename T, int D>
+template <typename T, int D, bool NS>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_ksel, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_vsel, const __grid_constant__ CUtensorMap tm_kcn,
                      const __grid_constant__ CUtensorMap tm_vcn, const AttnParams p) {
   using C = Cfg<T, D>;
+  static_assert(!NS || !C::kVT, "exact key blocks inside the Taylor path need bf16 tiles");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
@@ -276,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kv_it = 0, n_local = 0, k_issued = 0, v_issued = 0, q_arm0 = 0, q_arm1 = 0;
       bool ok = true;
       for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x, ++n_local) {
-        const Item it = decode_item(p, g);
+        const Item it = decode_item<NS>(p, g);
         if (n_local > 0 && !mbar_wait(&bars->q_empty, (n_local - 1) & 1)) {
           raise_abort(bars, p.err, kErrProducer);
           ok = false;
@@ -297,20 +345,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                           y, it.bh);
           }
         }
+        BlockCursor cur;
         for (int j = 0; j < it.nkv; ++j, ++kv_it) {
           if (aborted(bars)) { ok = false; break; }
           const int st = kv_it % C::STAGES;
           const uint32_t ph = (kv_it / C::STAGES) & 1;
+          // rows of K_new (or of the pooled rows) of the tile's two 64-row halves
+          int hrow0 = j * kBN, hrow1 = j * kBN + 64;
+          bool new_rows = it.kind == 0;
+          if constexpr (NS) {
+            if (j >= p.npt) {
+              new_rows = true;
+              if (p.b == 128) {
+                hrow0 = cur.next(p, it) * 128;
+                hrow1 = hrow0 + 64;
+              } else {
+                const int b0 = cur.next(p, it);
+                const int b1 = 2 * (j - p.npt) + 1 < it.nu ? cur.next(p, it) : b0;  // missing: masked
+                hrow0 = b0 * 64;
+                hrow1 = b1 * 64;
+              }
+            }
+          }
           // K tile
           if (!mbar_wait(&bars->k_empty[st], ph ^ 1)) { raise_abort(bars, p.err, kErrProducer); ok = false; break; }
           mbar_arrive_expect_tx(&bars->k_full[st], C::TILE);
           ++k_issued;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int r0 = j * kBN + 64 * h;
+            const int r0 = h ? hrow1 : hrow0;
             const CUtensorMap* map;
             int y;
-            if (it.kind == 0) {
+            if (new_rows) {
               if (r0 < p.L_src) { map = &tm_k; y = r0; } else { map = &tm_ksel; y = r0 - p.L_src; }
             } else {
               map = &tm_kcn; y = r0;
@@ -334,10 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int r0 = j * kBN + 64 * h;
+              const int r0 = h ? hrow1 : hrow0;
               const CUtensorMap* map;
               int y;
-              if (it.kind == 0) {
+              if (new_rows) {
                 if (r0 < p.L_src) { map = &tm_v; y = r0; } else { map = &tm_vsel; y = r0 - p.L_src; }
               } else {
                 map = &tm_vcn; y = r0;
@@ -401,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x) {
-        const Item it = decode_item(p, g);
+        const Item it = decode_item<NS>(p, g);
         const bool two = it.ntiles > 1;
         if (!wait_or_abort(&bars->q_full[0], q_cnt0 & 1)) break;
         ++q_cnt0;
@@ -483,9 +549,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     T* out = static_cast<T*>(p.out);
     for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x) {
-      const Item it = decode_item(p, g);
+      const Item it = decode_item<NS>(p, g);
       if (t >= it.ntiles) continue;
       float m = -FLT_MAX, l = 0.f;
+      // NS: this row's query block and its exact-block bitmask
+      BlockCursor cur;
+      const uint32_t* own = nullptr;
+      if constexpr (NS) {
+        const int u = t * p.bpt + row / p.b;
+        own = p.nsmask + ((size_t)it.bh * p.n_q + it.blk(u < it.nblk ? u : 0)) * p.ns_words;
+      }
       for (int j = 0; j < it.nkv; ++j) {
         if (!warp_wait(bars, &bars->s_full[t], s_cnt & 1, p.err)) { ok = false; break; }
         ++s_cnt;
@@ -493,7 +566,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kCols / 32; ++c) tmem_ld32(t_s + 32 * c, r + 32 * c);
         tmem_ld_wait<kCols>(r);
-        if (j == it.nkv - 1 && it.last_valid < kBN) {  // ragged last K/V tile (uniform branch)
+        float bias = 0.f;  // log2 of the weight of this tile's keys
+        if constexpr (NS) {
+          constexpr uint32_t kNegInf = 0xff800000u;
+          if (j < p.npt) {
+            // pooled rows: weight b, the row's own exact blocks and the rows past n_new masked
+            bias = p.bias_log2;
+            const int lim = j == p.npt - 1 ? it.last_valid : kBN;
+#pragma unroll
+            for (int c = 0; c < kCols / 32; ++c) {
+              const int wd = (kCols / 32) * j + c;
+              const uint32_t mw = wd < p.ns_words ? __ldg(own + wd) : 0u;
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                r[32 * c + i] = (((mw >> i) & 1u) != 0u || 32 * c + i >= lim) ? kNegInf : r[32 * c + i];
+            }
+          } else {
+            // exact blocks of the union: keep those in the row's own set
+            bool keep0, keep1;
+            if (p.b == 128) {
+              const int bk = cur.next(p, it);
+              keep0 = keep1 = ((__ldg(own + (bk >> 5)) >> (bk & 31)) & 1u) != 0u;
+            } else {
+              const int b0 = cur.next(p, it);
+              keep0 = ((__ldg(own + (b0 >> 5)) >> (b0 & 31)) & 1u) != 0u;
+              keep1 = false;
+              if (2 * (j - p.npt) + 1 < it.nu) {
+                const int b1 = cur.next(p, it);
+                keep1 = ((__ldg(own + (b1 >> 5)) >> (b1 & 31)) & 1u) != 0u;
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < kCols; ++i) r[i] = (i < kCols / 2 ? keep0 : keep1) ? r[i] : kNegInf;
+          }
+        } else if (j == it.nkv - 1 && it.last_valid < kBN) {  // ragged last K/V tile (uniform branch)
 #pragma unroll
           for (int i = 0; i < kCols; ++i)
             if (i >= it.last_valid) r[i] = __float_as_uint(-INFINITY);
@@ -508,7 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 8; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[i + c]), __uint_as_float(r[i + 8 + c]));
         }
         const float mx = fmaxf(fmax3(mc[0], mc[1], mc[2]), fmax3(fmax3(mc[3], mc[4], mc[5]), mc[6], mc[7])) *
-                         p.scale_log2;
+                             p.scale_log2 +
+                         bias;
         // lazy max: move it only when the tile's max exceeds it by more than 2^8
         const bool need = (j > 0) && (mx > m + kRescaleThreshold);
         const float alpha = need ? ex2_approx(m - mx) : 1.0f;
@@ -532,7 +639,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // p = 2^(s * scale - m), in pairs (pairs with i % kPolyDen < kPolyNum on the FMA
         // pipe, the rest on ex2). P is written and released in two halves (keys 0-63,
         // then 64-127) so that the P V MMAs can start on the first half.
-        const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(-m, -m);
+        // NS: a row with no unmasked key yet has m = -inf and all its entries -inf (p = 0)
+        const float nm = (NS && m == -INFINITY) ? 0.f : bias - m;
+        const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(nm, nm);
         uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -598,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool NS>
 cudaError_t launch_t(const void* q, const void* k, const void* v, void* out, const Plan& pl, const Work& w,
                      cudaStream_t s, int* n_ctas) {
   using C = Cfg<T, D>;
@@ -617,10 +726,15 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, void* out, con
   p.n_new = pl.n_new;
   p.bpt = kBM / pl.b;
   p.bpi = 2 * p.bpt;
-  p.items_e = (pl.n_exact + p.bpi - 1) / p.bpi;
+  p.items_e = NS ? 0 : (pl.n_exact + p.bpi - 1) / p.bpi;  // NS: Taylor items only
   p.items_t = (pl.n_flat + p.bpi - 1) / p.bpi;
   p.total = pl.BH * (p.items_e + p.items_t);
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  p.nsmask = w.nsmask;
+  p.ns_words = pl.ns_words;
+  p.npt = (pl.n_new + kBN - 1) / kBN;
+  p.bias_log2 = log2f((float)pl.b);
+  if (NS && (pl.k_ns <= 0 || w.nsmask == nullptr)) return cudaErrorInvalidValue;
   if (n_ctas) *n_ctas = 0;
   if (p.total == 0) return cudaSuccess;
 
@@ -642,7 +756,7 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, void* out, con
   }
   if (!ok) return cudaErrorInvalidValue;
 
-  auto kern = attention_kernel<T, D>;
+  auto kern = attention_kernel<T, D, NS>;
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
@@ -661,10 +775,17 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, void* out, con
 
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out, const Plan& p, const Work& w,
                              cudaStream_t s, int* n_ctas) {
-  if (p.dt == 0) return p.D == 128 ? launch_t<__nv_bfloat16, 128>(q, k, v, out, p, w, s, n_ctas)
-                                   : launch_t<__nv_bfloat16, 64>(q, k, v, out, p, w, s, n_ctas);
-  if (p.D == 64) return launch_t<float, 64>(q, k, v, out, p, w, s, n_ctas);
+  if (p.dt == 0) return p.D == 128 ? launch_t<__nv_bfloat16, 128, false>(q, k, v, out, p, w, s, n_ctas)
+                                   : launch_t<__nv_bfloat16, 64, false>(q, k, v, out, p, w, s, n_ctas);
+  if (p.D == 64) return launch_t<float, 64, false>(q, k, v, out, p, w, s, n_ctas);
   return cudaErrorNotSupported;
+}
+
+cudaError_t launch_attention_ns(const void* q, const void* k, const void* v, void* out, const Plan& p,
+                                const Work& w, cudaStream_t s) {
+  if (p.dt != 0) return cudaErrorNotSupported;
+  return p.D == 128 ? launch_t<__nv_bfloat16, 128, true>(q, k, v, out, p, w, s, nullptr)
+                    : launch_t<__nv_bfloat16, 64, true>(q, k, v, out, p, w, s, nullptr);
 }
 
 }  // namespace isa

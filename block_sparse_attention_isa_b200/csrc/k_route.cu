@@ -20,6 +20,13 @@
 // its rows, and its share of the pooled K_new / V_new rows in the attention
 // kernel's element type. The last CTA of a head sorts (M_i, i), then writes the
 // route list: exact blocks ascending followed by Taylor blocks ascending.
+//
+// With k_ns > 0 (the no-sparsity ratio alpha_ns of papernotes.org, Key design 3)
+// each row also picks the k_ns blocks of K_new with the largest coarse scores
+// (ties to the lower index) from the same scores: the k_ns-th largest score is
+// found by a bitwise search over order-preserving integer keys (32 counting
+// passes over the row), then the blocks above it and the first equal ones are
+// written as an ascending list and as a bitmask over K_new's blocks.
 #include <cuda_bf16.h>
 #include <float.h>
 
@@ -35,6 +42,44 @@ constexpr int kGroups = kThreads / kKeys;  // row groups
 
 __device__ __forceinline__ void store_elem(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void store_elem(float* p, float x) { *p = x; }
+
+// Unsigned key with the order of the float (-0 folded into +0; no NaN inputs).
+__device__ __forceinline__ uint32_t order_key(float x) {
+  const uint32_t u = __float_as_uint(x + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The k_ns largest entries of one row (ties to the lower index), by one warp:
+// ascending list into nsel[k_ns], bitmask into nsmask[ceil(n / 32)].
+__device__ __forceinline__ void select_row_blocks(const float* row, int n, int k_ns, int lane, int32_t* nsel,
+                                                  uint32_t* nsmask) {
+  uint32_t t = 0;  // grows to the key of the k_ns-th largest entry
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = t | (1u << bit);
+    int c = 0;
+    for (int j = lane; j < n; j += 32) c += order_key(row[j]) >= cand ? 1 : 0;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (c >= k_ns) t = cand;
+  }
+  int above = 0;
+  for (int j = lane; j < n; j += 32) above += order_key(row[j]) > t ? 1 : 0;
+  above = __reduce_add_sync(0xffffffffu, above);
+  int eq_left = k_ns - above;  // entries equal to the threshold still to take, lowest index first
+  int pos = 0;
+  const uint32_t below = (1u << lane) - 1u;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < n ? order_key(row[j]) : 0u;
+    const bool eq = j < n && key == t;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const bool take = (j < n && key > t) || (eq && __popc(eqm & below) < eq_left);
+    eq_left = max(0, eq_left - __popc(eqm));
+    const uint32_t tm = __ballot_sync(0xffffffffu, take);
+    if (lane == 0) nsmask[j0 >> 5] = tm;
+    if (take) nsel[pos + __popc(tm & below)] = j;
+    pos += __popc(tm);
+  }
+}
 
 template <int D>
 __host__ __device__ constexpr int key_stride() { return D + 4; }  // floats; 4-word skew between consecutive key rows
@@ -123,6 +168,13 @@ __global__ void __launch_bounds__(kThreads) route_kernel(Plan p, Work w) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) w.sharp[(size_t)bh * n_q + i0 + r] = v * inv_n;
+  }
+  if (p.k_ns > 0) {
+#pragma unroll 1
+    for (int r = warp; r < nr; r += kThreads / 32) {
+      const size_t gi = (size_t)bh * n_q + i0 + r;
+      select_row_blocks(lg + r * n_new, n_new, p.k_ns, lane, w.nsel + gi * p.k_ns, w.nsmask + gi * p.ns_words);
+    }
   }
 
   // pooled K_new / V_new rows for the Taylor path, in the MMA element type

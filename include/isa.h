@@ -197,6 +197,46 @@ ISA_API int isa_select_context_noalloc(const void* q, const void* k, const void*
 /* Number of kernel launches one isa_forward_ex call makes for these sizes (0 if invalid). */
 ISA_API int isa_launch_count(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, isa_dtype dt);
 
+/*
+ * No-sparsity ratio alpha_ns (papernotes.org, Key design 3; the notes quote
+ * alpha_ns = 0.0625, i.e. 93.75 % sparsity inside the Taylor path). Inside
+ * every Taylor-path query block i, the k_ns = ceil(alpha_ns * n_new - 1e-4)
+ * blocks of K_new with the largest coarse scores softmax(Qc_i Kc_new^T /
+ * sqrt(D)) (ties to the lower block index) are computed exactly, key by key;
+ * the other blocks stay pooled with weight b (papernotes.org, Key design 2:
+ * l += P^c * b, O += P^c Vc * b), and one softmax covers both kinds of terms.
+ * With alpha_ns = 0 every call below equals its plain counterpart. Needs
+ * bfloat16 inputs when alpha_ns > 0 (ISA_ERR_UNSUPPORTED otherwise).
+ */
+
+/* isa_plan with alpha_ns: also writes k_ns (exact key blocks per Taylor query block). */
+ISA_API int isa_plan_ns(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f,
+                        float alpha_ns, int32_t* n_q, int32_t* k, int32_t* n_flat, int32_t* k_ns);
+
+/* isa_workspace_bytes with alpha_ns: adds the per-query-block lists and bitmasks of exact key blocks. */
+ISA_API size_t isa_workspace_bytes_ns(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s,
+                                      float alpha_ns, isa_dtype dt);
+
+/*
+ * isa_forward_ns - isa_forward_ex with the no-sparsity ratio alpha_ns in [0, 1].
+ * Arguments, layout, ownership and errors as for isa_forward_ex, plus:
+ *   dbg_ns       optional device int32 [B, H, n_q, k_ns]: for every query block
+ *                (in block order) its exactly computed K_new blocks, ascending
+ *                (0-based blocks of K_new: source blocks, then kept context
+ *                blocks in K_new order); written for Taylor and exact query
+ *                blocks alike, used only by the Taylor ones; NULL to skip
+ *   workspace    at least isa_workspace_bytes_ns() bytes
+ * With alpha_ns > 0 the Taylor query blocks take one extra kernel launch.
+ */
+ISA_API int isa_forward_ns(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D,
+                           int b, float alpha_s, float alpha_f, float alpha_ns, isa_dtype dt, void* out,
+                           int32_t* dbg_sel, int32_t* dbg_route, int32_t* dbg_ns, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Number of kernel launches one isa_forward_ns call makes for these sizes (0 if invalid). */
+ISA_API int isa_launch_count_ns(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f,
+                                float alpha_ns, isa_dtype dt);
+
 /* Message of the last failed call on this host thread ("" if none). */
 ISA_API const char* isa_last_error(void);
 

@@ -52,9 +52,9 @@ the design notes):
 * Each query block takes exactly one path, so write-back is a scatter into
   the original token order with no merge.
 * The Taylor path is computed literally, with the block-length weight b.
-* No-sparsity ratio alpha_ns (papernotes.org, "Key design 2" block mask M_ij
-  and "Key design 3" "alpha_ns controls the in-block non-sparse share";
-  paperlayer.ai summary section 2 "Pooling Attention": top-k entries of the
+* No-sparsity ratio alpha_ns (papernotes.org, "Key design 2" block mask M_ij;
+  "Key design 3": alpha_ns sets the share of key blocks that stay dense inside
+  a Taylor query block; paperlayer.ai summary section 2 "Pooling Attention": top-k entries of the
   coarse map give the block mask; section 4 defaults alpha_ns = 0.0625). For
   a Taylor query block i, the k_ns = ceil(alpha_ns * n_new - 1e-4) key blocks
   of K_new with the largest coarse scores softmax_j(Qc_i . Kc_new_j / sqrt(D))
@@ -338,7 +338,9 @@ def isa_select_route_ref(q: np.ndarray, k: np.ndarray, L_src: int, L_ctx: int, b
     return dict(qc=qc, kc=kc, s_coarse=s_coarse, colscore=colscore, sel=sel, kc_new=k_new_pooled,
                 sharp=m, exact=exact, taylor=taylor, k=kk, n_flat=n_flat, k_ns=k_ns, ns_sel=ns_sel,
                 topk_margin=topk_margin(colscore, kk), route_margin=route_margin(m, n_flat),
-                ns_margin=no_sparse_margin(p_new[taylor], k_ns) if k_ns else float("inf"))
+                ns_margin=no_sparse_margin(p_new[taylor], k_ns) if k_ns else float("inf"),
+                ns_row_margin=np.array([no_sparse_margin(p_new[[i]], k_ns) for i in range(n_q)]) if k_ns
+                else np.full(n_q, np.inf))
 
 
 def isa_slice_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, L_src: int, L_ctx: int, b: int,
