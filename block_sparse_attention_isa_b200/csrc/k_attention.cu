@@ -42,8 +42,10 @@
 // their one softmax). Each query block u has its own set E_u of k_ns blocks of
 // K_new. An item (the Taylor blocks of two query tiles) walks first the pooled
 // rows of K_new, each weighted by b (a log2(b) bias on its exponent) and masked
-// for the row's own E_u, then the key tiles of the union of its blocks' E_u,
-// where every row masks the blocks outside its own E_u.
+// for the row's own E_u, then the key tiles of the union of its blocks' E_u.
+// The K/V tiles are loaded once for both query tiles, but a query tile takes
+// part (S and P V MMAs, softmax) only in the key tiles that hold one of its own
+// blocks' E_u; inside those, every row masks the blocks outside its own E_u.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 #include <float.h>
@@ -118,6 +120,9 @@ struct Bars {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  // NS: query tiles taking part in the K/V tile of each stage (bit t = tile t), written by
+  // the producer before it arms k_full of the stage, read by the MMA issuer after that wait
+  uint32_t stage_tiles[2];
 };
 
 template <typename T, int D>
@@ -180,6 +185,34 @@ struct BlockCursor {
     return 32 * wd + j;
   }
 };
+
+// NS: blocks of exact K/V tile j (the next 128 / b blocks of the union); bk1 is the
+// second 64-key block when b = 64, or -1 (b = 128, or past the end of the union).
+struct KeyTile {
+  int bk0, bk1;
+};
+__device__ __forceinline__ KeyTile next_key_tile(const AttnParams& p, const Item& it, BlockCursor& cur, int j) {
+  KeyTile kt;
+  kt.bk0 = cur.next(p, it);
+  kt.bk1 = (p.b == 64 && 2 * (j - p.npt) + 1 < it.nu) ? cur.next(p, it) : -1;
+  return kt;
+}
+__device__ __forceinline__ bool has_block(const uint32_t* mask, int bk) {
+  return bk >= 0 && ((__ldg(mask + (bk >> 5)) >> (bk & 31)) & 1u) != 0u;
+}
+
+template <bool NS>
+__device__ __forceinline__ Item decode_item(const AttnParams& p, int g);
+
+// NS: whether query tile t of the item keeps a block of the K/V tile (any of its query blocks)
+__device__ __forceinline__ bool tile_keeps(const AttnParams& p, const Item& it, int t, const KeyTile& kt) {
+  const int u0 = t * p.bpt, u1 = min(it.nblk, u0 + p.bpt);
+  for (int u = u0; u < u1; ++u) {
+    const uint32_t* m = p.nsmask + ((size_t)it.bh * p.n_q + it.blk(u)) * p.ns_words;
+    if (has_block(m, kt.bk0) || has_block(m, kt.bk1)) return true;
+  }
+  return false;
+}
 
 template <bool NS>
 __device__ __forceinline__ Item decode_item(const AttnParams& p, int g) {
@@ -353,22 +386,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           // rows of K_new (or of the pooled rows) of the tile's two 64-row halves
           int hrow0 = j * kBN, hrow1 = j * kBN + 64;
           bool new_rows = it.kind == 0;
+          uint32_t tiles = 3u;  // NS: query tiles taking part in this K/V tile
           if constexpr (NS) {
             if (j >= p.npt) {
               new_rows = true;
+              const KeyTile kt = next_key_tile(p, it, cur, j);
+              tiles = (tile_keeps(p, it, 0, kt) ? 1u : 0u) | (it.ntiles > 1 && tile_keeps(p, it, 1, kt) ? 2u : 0u);
               if (p.b == 128) {
-                hrow0 = cur.next(p, it) * 128;
+                hrow0 = kt.bk0 * 128;
                 hrow1 = hrow0 + 64;
               } else {
-                const int b0 = cur.next(p, it);
-                const int b1 = 2 * (j - p.npt) + 1 < it.nu ? cur.next(p, it) : b0;  // missing: masked
-                hrow0 = b0 * 64;
-                hrow1 = b1 * 64;
+                hrow0 = kt.bk0 * 64;
+                hrow1 = (kt.bk1 >= 0 ? kt.bk1 : kt.bk0) * 64;  // missing second block: loaded, masked
               }
             }
           }
           // K tile
           if (!mbar_wait(&bars->k_empty[st], ph ^ 1)) { raise_abort(bars, p.err, kErrProducer); ok = false; break; }
+          if constexpr (NS) *reinterpret_cast<volatile uint32_t*>(&bars->stage_tiles[st]) = tiles;
           mbar_arrive_expect_tx(&bars->k_full[st], C::TILE);
           ++k_issued;
 #pragma unroll
@@ -475,6 +510,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!wait_or_abort(&bars->q_full[1], q_cnt1 & 1)) break;
           ++q_cnt1;
         }
+        // NS: the query tiles taking part in this step and the next (the first K/V tile holds
+        // pooled rows, in which every query tile takes part)
+        bool pc0 = true, pc1 = two;
         // S_t for the first K/V tile
         {
           const uint32_t st = kv_it % C::STAGES;
@@ -491,42 +529,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int j = 0; j < it.nkv; ++j, ++kv_it) {
           const uint32_t st = kv_it % C::STAGES;
-          if (!wait_or_abort(&bars->v_full[st], (kv_it / C::STAGES) & 1)) break;
           const bool more = (j + 1 < it.nkv);
+          bool pn0 = more, pn1 = more && two;  // NS: read from the stage once it is full
+          if (!wait_or_abort(&bars->v_full[st], (kv_it / C::STAGES) & 1)) break;
           const uint32_t st1 = (kv_it + 1) % C::STAGES;
           const uint32_t va = st ? v_lo1 : v_lo0;
           const uint32_t ka1 = st1 ? k_lo1 : k_lo0;
           const uint32_t acc = j > 0 ? 1u : 0u;
           // tile 0: P0 V_j in two halves (each as soon as its P is written), then S0 of the next K/V tile
-          if (!wait_or_abort(&bars->p_half[0][0], pv_cnt0 & 1)) break;
-          issue_pv(t_o0, t_s0, va, acc, 0);
-          if (!wait_or_abort(&bars->p_half[0][1], pv_cnt0 & 1)) break;
-          issue_pv(t_o0, t_s0, va, 1u, 1);
-          umma_commit(&bars->o_done[0]);
-          ++pv_cnt0;
+          if (!NS || pc0) {
+            if (!wait_or_abort(&bars->p_half[0][0], pv_cnt0 & 1)) break;
+            issue_pv(t_o0, t_s0, va, acc, 0);
+            if (!wait_or_abort(&bars->p_half[0][1], pv_cnt0 & 1)) break;
+            issue_pv(t_o0, t_s0, va, 1u, 1);
+            umma_commit(&bars->o_done[0]);
+            ++pv_cnt0;
+          }
           if (more) {
             if (!wait_or_abort(&bars->k_full[st1], ((kv_it + 1) / C::STAGES) & 1)) break;
-            issue_s(t_s0, q_lo0, ka1);
-            umma_commit(&bars->s_full[0]);
+            if constexpr (NS) {
+              const uint32_t tiles = *reinterpret_cast<volatile uint32_t*>(&bars->stage_tiles[st1]);
+              pn0 = (tiles & 1u) != 0u;
+              pn1 = two && (tiles & 2u) != 0u;
+            }
+            if (!NS || pn0) {
+              issue_s(t_s0, q_lo0, ka1);
+              umma_commit(&bars->s_full[0]);
+            }
           }
           // tile 1
-          if (two) {
+          if (NS ? pc1 : two) {
             if (!wait_or_abort(&bars->p_half[1][0], pv_cnt1 & 1)) break;
             issue_pv(t_o1, t_s1, va, acc, 0);
             if (!wait_or_abort(&bars->p_half[1][1], pv_cnt1 & 1)) break;
             issue_pv(t_o1, t_s1, va, 1u, 1);
             umma_commit(&bars->o_done[1]);
             ++pv_cnt1;
-            if (more) {
-              issue_s(t_s1, q_lo1, ka1);
-              umma_commit(&bars->s_full[1]);
-            }
+          }
+          if (NS ? pn1 : (two && more)) {
+            issue_s(t_s1, q_lo1, ka1);
+            umma_commit(&bars->s_full[1]);
           }
           if (more) {
             umma_commit(&bars->k_empty[st1]);
             if (j + 2 == it.nkv) umma_commit(&bars->q_empty);
           }
           umma_commit(&bars->v_empty[st]);
+          pc0 = pn0;
+          pc1 = pn1;
         }
       }
       // every MMA issued by this thread completes before TMEM can be released
@@ -560,6 +610,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         own = p.nsmask + ((size_t)it.bh * p.n_q + it.blk(u < it.nblk ? u : 0)) * p.ns_words;
       }
       for (int j = 0; j < it.nkv; ++j) {
+        bool keep0 = true, keep1 = true;  // NS: this row keeps the K/V tile's first / second 64 keys
+        if constexpr (NS) {
+          if (j >= p.npt) {
+            const KeyTile kt = next_key_tile(p, it, cur, j);
+            if (!tile_keeps(p, it, t, kt)) continue;  // no row of this tile keeps the K/V tile
+            keep0 = has_block(own, kt.bk0);
+            keep1 = p.b == 128 ? keep0 : has_block(own, kt.bk1);
+          }
+        }
         if (!warp_wait(bars, &bars->s_full[t], s_cnt & 1, p.err)) { ok = false; break; }
         ++s_cnt;
         uint32_t r[kCols];
@@ -583,19 +642,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
             // exact blocks of the union: keep those in the row's own set
-            bool keep0, keep1;
-            if (p.b == 128) {
-              const int bk = cur.next(p, it);
-              keep0 = keep1 = ((__ldg(own + (bk >> 5)) >> (bk & 31)) & 1u) != 0u;
-            } else {
-              const int b0 = cur.next(p, it);
-              keep0 = ((__ldg(own + (b0 >> 5)) >> (b0 & 31)) & 1u) != 0u;
-              keep1 = false;
-              if (2 * (j - p.npt) + 1 < it.nu) {
-                const int b1 = cur.next(p, it);
-                keep1 = ((__ldg(own + (b1 >> 5)) >> (b1 & 31)) & 1u) != 0u;
-              }
-            }
 #pragma unroll
             for (int i = 0; i < kCols; ++i) r[i] = (i < kCols / 2 ? keep0 : keep1) ? r[i] : kNegInf;
           }

@@ -25,8 +25,9 @@
 // each row also picks the k_ns blocks of K_new with the largest coarse scores
 // (ties to the lower index) from the same scores: the k_ns-th largest score is
 // found by a bitwise search over order-preserving integer keys (32 counting
-// passes over the row), then the blocks above it and the first equal ones are
-// written as an ascending list and as a bitmask over K_new's blocks.
+// passes over the row, held in registers when n_new <= 256), then the blocks
+// above it and the first equal ones are written as an ascending list and as a
+// bitmask over K_new's blocks.
 #include <cuda_bf16.h>
 #include <float.h>
 
@@ -50,7 +51,43 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 }
 
 // The k_ns largest entries of one row (ties to the lower index), by one warp:
-// ascending list into nsel[k_ns], bitmask into nsmask[ceil(n / 32)].
+// ascending list into nsel[k_ns], bitmask into nsmask[ceil(n / 32)]. Rows of up to
+// 32 * KPL entries keep their keys in registers (entry lane + 32 i in key[i]).
+template <int KPL>
+__device__ __forceinline__ void select_row_blocks_reg(const float* row, int n, int k_ns, int lane, int32_t* nsel,
+                                                      uint32_t* nsmask) {
+  uint32_t key[KPL];  // 0 past the end: every real key is above 0
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) key[i] = lane + 32 * i < n ? order_key(row[lane + 32 * i]) : 0u;
+  uint32_t t = 0;  // grows to the key of the k_ns-th largest entry
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = t | (1u << bit);
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) c += key[i] >= cand ? 1 : 0;
+    if (__reduce_add_sync(0xffffffffu, c) >= k_ns) t = cand;
+  }
+  int above = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) above += key[i] > t ? 1 : 0;
+  int eq_left = k_ns - __reduce_add_sync(0xffffffffu, above);
+  int pos = 0;
+  const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    if (32 * i >= n) break;
+    const bool eq = key[i] == t;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const bool take = key[i] > t || (eq && __popc(eqm & below) < eq_left);
+    eq_left = max(0, eq_left - __popc(eqm));
+    const uint32_t tm = __ballot_sync(0xffffffffu, take);
+    if (lane == 0) nsmask[i] = tm;
+    if (take) nsel[pos + __popc(tm & below)] = lane + 32 * i;
+    pos += __popc(tm);
+  }
+}
+
+// The same for rows of any length, reading the keys from shared memory on every pass.
 __device__ __forceinline__ void select_row_blocks(const float* row, int n, int k_ns, int lane, int32_t* nsel,
                                                   uint32_t* nsmask) {
   uint32_t t = 0;  // grows to the key of the k_ns-th largest entry
@@ -173,7 +210,11 @@ __global__ void __launch_bounds__(kThreads) route_kernel(Plan p, Work w) {
 #pragma unroll 1
     for (int r = warp; r < nr; r += kThreads / 32) {
       const size_t gi = (size_t)bh * n_q + i0 + r;
-      select_row_blocks(lg + r * n_new, n_new, p.k_ns, lane, w.nsel + gi * p.k_ns, w.nsmask + gi * p.ns_words);
+      if (n_new <= 256)
+        select_row_blocks_reg<8>(lg + r * n_new, n_new, p.k_ns, lane, w.nsel + gi * p.k_ns,
+                                 w.nsmask + gi * p.ns_words);
+      else
+        select_row_blocks(lg + r * n_new, n_new, p.k_ns, lane, w.nsel + gi * p.k_ns, w.nsmask + gi * p.ns_words);
     }
   }
 
