@@ -110,3 +110,58 @@ def test_launch_count(L):
 def test_host_entry_rejects_before_copying(L):
     assert L.isa_forward_host(None, FAKE, FAKE, 1, 1, 64, 64, 64, 64, 0.5, 0.5, 0, FAKE + 4096, None, None) == -1
     assert L.isa_forward_host(FAKE, FAKE, FAKE, 1, 1, 64, 60, 64, 64, 0.5, 0.5, 0, FAKE + (1 << 30), None, None) == -2
+
+
+# ---------------------------------------------------------------- no-sparsity ratio alpha_ns
+
+@pytest.mark.parametrize("a_ns", [0.0, 0.01, 0.0625, 0.1, 0.125, 0.3, 0.5, 0.999, 1.0])
+@pytest.mark.parametrize("name", ["tiny_f32_n1024", "bf16_n8192_b64", "bf16_n32768_b128",
+                                  "bf16_n51200_b128_as0.1_af0.3_sc0.5"])
+def test_no_sparse_count_matches_oracle(L, name, a_ns):
+    """k_ns of the C plan equals the oracle's count and the bench's FLOP-count helper."""
+    import bench
+    w = isa_synth.all_workloads()[name]
+    n_q, k, n_flat, k_ns = isa.plan_ns(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, w.alpha_f, a_ns)
+    assert (n_q, k, n_flat) == isa.plan(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, w.alpha_f)
+    n_new = w.L_src // w.b + k
+    assert k_ns == O.no_sparse_block_count(a_ns, n_new) == bench.no_sparse_count(a_ns, n_new)
+
+
+def test_alpha_ns_sizes_and_launches(L):
+    args = (1, 40, 16384, 16384, 128, 128, 0.25)
+    assert isa.plan_ns(*args, 0.6, 0.0625) == (256, 32, 153, 10)
+    # the exact-block lists (int32 [BH, n_q, k_ns]) and bitmasks (uint32 [BH, n_q, ceil(n_new / 32)])
+    extra = 40 * 256 * 10 * 4 + 40 * 256 * 5 * 4
+    assert isa.workspace_bytes(*args, alpha_ns=0.0625) - isa.workspace_bytes(*args) == extra
+    assert isa.workspace_bytes(*args, alpha_ns=0.0) == isa.workspace_bytes(*args)
+    assert isa.launch_count(*args, 0.6, alpha_ns=0.0625) == 5
+    assert isa.launch_count(*args, 0.6, alpha_ns=0.0) == 4
+    assert isa.launch_count(*args, 0.0, alpha_ns=0.0625) == 4  # no Taylor query block: no extra launch
+
+
+def _fwd_ns(L, a_ns, dt=0, D=64, ws=None, ws_bytes=0):
+    return L.isa_forward_ns(FAKE, FAKE + (1 << 33), FAKE + (2 << 33), 1, 2, 512, 512, D, 64, 0.5, 0.5, a_ns, dt,
+                            FAKE + (3 << 33), None, None, None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("a_ns,dt,code", [
+    (1.5, 0, -1), (-0.1, 0, -1), (float("nan"), 0, -1),
+    (0.1, 1, -3),   # float32 inputs with alpha_ns > 0
+    (0.0, 1, -4),   # float32 with alpha_ns = 0 is the plain pass: fails only for the missing workspace
+    (0.1, 0, -4),
+])
+def test_alpha_ns_argument_errors(L, a_ns, dt, code):
+    assert _fwd_ns(L, a_ns, dt) == code
+    assert isa.last_error() != ""
+
+
+def test_bench_flops_with_alpha_ns():
+    """Taylor FLOPs: each flat query row attends to n_new - k_ns pooled rows and k_ns * b keys."""
+    import bench
+    w = isa_synth.WORKLOADS["bf16_n32768_b128"]
+    f0, f1 = bench.flops_per_call(w), bench.flops_per_call(w, 0.0625)
+    assert f0 == bench.flops_per_call(w, 0.0)
+    per = 4.0 * 153 * 128 * 128 * w.H  # 4 * n_flat * b * D * BH
+    assert f0["taylor"] == per * 160
+    assert f1["taylor"] == per * (150 + 10 * 128)
+    assert f1["exact"] == f0["exact"] and f1["total"] - f0["total"] == f1["taylor"] - f0["taylor"]
