@@ -167,10 +167,11 @@ struct Item {
 };
 
 // NS: word `wd` of the union of the exact-block bitmasks of the item's query blocks
+// (blocks past nblk repeat blk0, so all loads are issued unconditionally and at once)
 __device__ __forceinline__ uint32_t union_word(const AttnParams& p, const Item& it, int wd) {
   const uint32_t* m = p.nsmask + (size_t)it.bh * p.n_q * p.ns_words + wd;
-  uint32_t x = 0;
-  for (int u = 0; u < it.nblk; ++u) x |= __ldg(m + (size_t)it.blk(u) * p.ns_words);
+  uint32_t x = __ldg(m + (size_t)it.blk0 * p.ns_words) | __ldg(m + (size_t)it.blk1 * p.ns_words);
+  if (p.bpi > 2) x |= __ldg(m + (size_t)it.blk2 * p.ns_words) | __ldg(m + (size_t)it.blk3 * p.ns_words);
   return x;
 }
 
@@ -248,8 +249,24 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p, int g) {
   it.ntiles = (it.nblk + p.bpt - 1) / p.bpt;
   if constexpr (NS) {
     // pooled rows, then the union of the exact blocks, 128 / b blocks per K/V tile
+    // (four words of every query block's mask per round, all loads issued before any is used;
+    // blocks past nblk repeat blk0, so OR-ing them changes nothing)
+    const uint32_t* m = p.nsmask + (size_t)it.bh * p.n_q * p.ns_words;
+    const uint32_t *m0 = m + (size_t)it.blk0 * p.ns_words, *m1 = m + (size_t)it.blk1 * p.ns_words;
+    const uint32_t *m2 = m + (size_t)it.blk2 * p.ns_words, *m3 = m + (size_t)it.blk3 * p.ns_words;
+    const bool four = p.bpi > 2;
     int nu = 0;
-    for (int wd = 0; wd < p.ns_words; ++wd) nu += __popc(union_word(p, it, wd));
+    for (int wd = 0; wd < p.ns_words; wd += 4) {
+      uint32_t x[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int w = min(wd + i, p.ns_words - 1);
+        x[i] = __ldg(m0 + w) | __ldg(m1 + w);
+        if (four) x[i] |= __ldg(m2 + w) | __ldg(m3 + w);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) nu += wd + i < p.ns_words ? __popc(x[i]) : 0;
+    }
     it.nu = nu;
     it.nkv = p.npt + (nu + p.bpt - 1) / p.bpt;
     it.last_valid = p.n_new - kBN * (p.npt - 1);  // of the last pooled tile
