@@ -165,3 +165,13 @@ def test_bench_flops_with_alpha_ns():
     assert f0["taylor"] == per * 160
     assert f1["taylor"] == per * (150 + 10 * 128)
     assert f1["exact"] == f0["exact"] and f1["total"] - f0["total"] == f1["taylor"] - f0["taylor"]
+
+
+def test_pass_roofline():
+    """(attention FLOPs / peak + pool and gather bytes / bandwidth), as a time and over the measured one."""
+    import bench
+    f = {"exact": 5.0e12, "taylor": 1.0e12}
+    hb = {"pool": 1.0e9, "gather": 0.5e9}
+    r = bench.pass_roofline(f, hb, ms=10.0, tflops=1000.0, gbs=5000.0)
+    assert abs(r["t_roof_ms"] - (6.0 + 0.3)) < 1e-9
+    assert abs(r["frac"] - 0.63) < 1e-12
