@@ -178,9 +178,8 @@ __device__ __forceinline__ uint32_t union_word(const AttnParams& p, const Item& 
 // NS: walks the union of an item's exact key blocks in ascending order. Callers ask
 // for at most it.nu blocks; past the end it returns block 0. (Walking the blocks that
 // only one query tile keeps in alternation, so that consecutive K/V tiles belong to
-// different tiles, measured slower: 6.39 ms against 5.88 ms for the attention stage
-// at the 32K-token workload with alpha_ns = 0.0625. Shorter steps leave the loads of
-// the two-stage K/V ring less time to land.)
+// different tiles, measured slower: 6.35 ms against 5.99 ms for the attention stage
+// at the 32K-token workload with alpha_ns = 0.0625, on one box.)
 struct BlockCursor {
   int wd = -1;
   uint32_t bits = 0;
@@ -207,9 +206,6 @@ __device__ __forceinline__ KeyTile next_key_tile(const AttnParams& p, const Item
 __device__ __forceinline__ bool has_block(const uint32_t* mask, int bk) {
   return bk >= 0 && ((__ldg(mask + (bk >> 5)) >> (bk & 31)) & 1u) != 0u;
 }
-
-template <bool NS>
-__device__ __forceinline__ Item decode_item(const AttnParams& p, int g);
 
 // NS: whether query tile t of the item keeps a block of the K/V tile (any of its query blocks)
 __device__ __forceinline__ bool tile_keeps(const AttnParams& p, const Item& it, int t, const KeyTile& kt) {
