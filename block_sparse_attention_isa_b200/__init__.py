@@ -299,13 +299,14 @@ def selftest_wait_timeout(workspace, timeout_ms: int = 100, stream=None):
 def debug_pooled(B, H, L_src, L_ctx, D, b, alpha_s, dtype=ISA_BF16, workspace=None, stream=None):
     """Intermediates of the last call made with ``workspace``: dict of Qc, Kc, Vc, colscore, sharp."""
     torch = _torch()
-    n_q = (L_src + L_ctx) // b
+    n_ctx = -(-L_ctx // b)                  # the last block of each part may be short
+    n_q = -(-L_src // b) + n_ctx
     dev = torch.cuda.current_device() if workspace is None else workspace.device
     if workspace is None:
         workspace = _WS_CACHE[dev]
     f = dict(device=workspace.device, dtype=torch.float32)
     res = dict(qc=torch.empty((B, H, n_q, D), **f), kc=torch.empty((B, H, n_q, D), **f),
-               vc=torch.empty((B, H, n_q, D), **f), colscore=torch.empty((B, H, L_ctx // b), **f),
+               vc=torch.empty((B, H, n_q, D), **f), colscore=torch.empty((B, H, n_ctx), **f),
                sharp=torch.empty((B, H, n_q), **f))
     if stream is None:
         stream = torch.cuda.current_stream(workspace.device)

@@ -65,14 +65,16 @@ int make_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, f
   if (D != 64 && D != 128) return fail(ISA_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
   if (b != 64 && b != 128) return fail(ISA_ERR_UNSUPPORTED, "block size b must be 64 or 128 (got %d)", b);
   if (dt == ISA_F32 && D != 64) return fail(ISA_ERR_UNSUPPORTED, "float32 inputs need D = 64");
-  if (L_src % b || L_ctx % b)
-    return fail(ISA_ERR_SHAPE, "L_src (%d) and L_ctx (%d) must be multiples of b (%d)", L_src, L_ctx, b);
   const long long N = (long long)L_src + L_ctx;
   if (N > (1ll << 30)) return fail(ISA_ERR_UNSUPPORTED, "N too large");
   const long long BH = (long long)B * H;
   if (BH > 65535) return fail(ISA_ERR_UNSUPPORTED, "B*H must be at most 65535");
-  const int n_q = (int)(N / b);
-  if (n_q > kMaxBlocks) return fail(ISA_ERR_UNSUPPORTED, "N / b must be at most %d (got %d)", kMaxBlocks, n_q);
+  // the source and the context part each end in a block of at most b tokens
+  const long long n_src = (L_src + (long long)b - 1) / b, n_ctx = (L_ctx + (long long)b - 1) / b;
+  const long long n_q_ll = n_src + n_ctx;
+  if (n_q_ll > kMaxBlocks)
+    return fail(ISA_ERR_UNSUPPORTED, "the block count must be at most %d (got %lld)", kMaxBlocks, n_q_ll);
+  const int n_q = (int)n_q_ll;
   p->B = B;
   p->H = H;
   p->BH = (int)BH;
@@ -82,11 +84,15 @@ int make_plan(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, f
   p->L_src = L_src;
   p->L_ctx = L_ctx;
   p->n_q = n_q;
-  p->n_src = L_src / b;
-  p->n_ctx = L_ctx / b;
+  p->n_src = (int)n_src;
+  p->n_ctx = (int)n_ctx;
   p->k = kept_blocks(alpha_s, p->n_ctx);
   p->n_new = p->n_src + p->k;
   p->L_new = p->n_new * b;
+  p->L_srcp = p->n_src * b;
+  p->len_src_last = L_src - (p->n_src - 1) * b;
+  p->len_ctx_last = L_ctx - (p->n_ctx - 1) * b;
+  p->ragged = (L_src % b || L_ctx % b) ? 1 : 0;
   p->n_flat = flat_blocks(alpha_f, n_q);
   p->n_exact = n_q - p->n_flat;
   p->dt = dt;

@@ -10,12 +10,16 @@ namespace isa {
 // Sizes of one call, all derived on the host from the arguments.
 struct Plan {
   int B, H, BH, N, D, b, L_src, L_ctx;
-  int n_q;     // N / b query blocks (also key blocks)
-  int n_src;   // L_src / b
-  int n_ctx;   // L_ctx / b
+  int n_q;     // n_src + n_ctx query blocks (also key blocks)
+  int n_src;   // ceil(L_src / b): source blocks from token 0, the last one possibly short
+  int n_ctx;   // ceil(L_ctx / b): context blocks from token L_src, the last one possibly short
   int k;       // kept context blocks
   int n_new;   // n_src + k blocks in K_new
-  int L_new;   // n_new * b keys in K_new
+  int L_new;   // n_new * b rows of K_new: every block takes b rows, a short one padded (masked)
+  int L_srcp;  // n_src * b: rows of the source part of K_new (rows L_src .. L_srcp - 1 masked)
+  int len_src_last;  // tokens of the last source block (b when b divides L_src)
+  int len_ctx_last;  // tokens of the last context block (b when b divides L_ctx)
+  int ragged;  // 1 when b does not divide L_src or L_ctx
   int n_flat;  // query blocks on the Taylor path
   int n_exact; // n_q - n_flat query blocks on the exact path
   int dt;      // 0 = bf16, 1 = fp32
@@ -23,6 +27,14 @@ struct Plan {
   int k_ns;    // key blocks of K_new computed exactly inside each Taylor query block (0: plain Taylor path)
   int ns_words;  // 32-bit words of one query block's exact-key-block bitmask (ceil(n_new / 32))
 };
+
+// First token of block i (source blocks from 0, context blocks from L_src) and its length.
+__host__ __device__ inline int block_start(const Plan& p, int i) {
+  return i < p.n_src ? i * p.b : p.L_src + (i - p.n_src) * p.b;
+}
+__host__ __device__ inline int block_len(const Plan& p, int i) {
+  return i == p.n_src - 1 ? p.len_src_last : (i == p.n_q - 1 ? p.len_ctx_last : p.b);
+}
 
 // Row length of the transposed pooled V rows (fp32 inputs): n_new rounded up to 4
 // floats so that the rows start on 16-byte boundaries, as TMA requires.

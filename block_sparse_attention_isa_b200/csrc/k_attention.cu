@@ -105,6 +105,11 @@ struct AttnParams {
   int ns_words;            // NS: ceil(n_new / 32)
   int npt;                 // NS: K/V tiles of the pooled rows, ceil(n_new / 128)
   float bias_log2;         // NS: log2(b), the weight of a pooled row in the exponent
+  // Short blocks (b does not divide L_src or L_ctx). Block j of K_new takes rows [j b, j b + b),
+  // the rows past a short block's length are masked; a pooled row weighs its block's length.
+  const int32_t* sel;      // [BH, k] kept context blocks (the short last one can only be the last kept)
+  int k, n_src, n_ctx, L_srcp, len_src_last, len_ctx_last, ragged;
+  float src_last_bias, ctx_last_bias;  // log2(len / b) / scale_log2: raw-score offsets of short pooled rows
   int BH, N, b, L_src, n_q, n_exact, n_flat, L_new, n_new;
   int bpt;       // blocks per 128-row tile (128 / b)
   int bpi;       // blocks per item (2 tiles)
@@ -113,6 +118,22 @@ struct AttnParams {
   int total;     // all items
   float scale_log2;
 };
+
+// First token of query block i (source blocks from 0, context blocks from L_src) and its length.
+__device__ __forceinline__ int qblock_start(const AttnParams& p, int i) {
+  return i < p.n_src ? i * p.b : p.L_src + (i - p.n_src) * p.b;
+}
+__device__ __forceinline__ int qblock_len(const AttnParams& p, int i) {
+  return i == p.n_src - 1 ? p.len_src_last : (i == p.n_q - 1 ? p.len_ctx_last : p.b);
+}
+// Whether head bh keeps the short last context block, which is then the last block of K_new.
+__device__ __forceinline__ bool short_ctx_kept(const AttnParams& p, int bh) {
+  return p.len_ctx_last < p.b && p.k > 0 && __ldg(p.sel + (size_t)bh * p.k + p.k - 1) == p.n_ctx - 1;
+}
+// Keys held by block j of K_new (b unless it is a short block).
+__device__ __forceinline__ int new_block_len(const AttnParams& p, int j, bool ctx_short) {
+  return j == p.n_src - 1 ? p.len_src_last : (ctx_short && j == p.n_new - 1 ? p.len_ctx_last : p.b);
+}
 
 struct Bars {
   uint64_t q_full[2];
@@ -294,6 +315,22 @@ __device__ __forceinline__ bool warp_wait(Bars* b, uint64_t* bar, uint32_t parit
   return ok;
 }
 
+// -inf on the scores of the K/V tile columns whose K_new rows (tile rows from `base`) lie in [lo, hi)
+__device__ __forceinline__ void mask_key_rows(uint32_t (&r)[kCols], int base, int lo, int hi) {
+  if (hi <= base || lo >= base + kBN) return;  // the same for every thread of the CTA
+#pragma unroll
+  for (int i = 0; i < kCols; ++i)
+    if (base + i >= lo && base + i < hi) r[i] = 0xff800000u;
+}
+// Adds `delta` to the raw score of the column holding pooled row `col` (tile rows from `base`)
+__device__ __forceinline__ void add_col_bias(uint32_t (&r)[kCols], int base, int col, float delta) {
+  const int c = col - base;
+  if (c < 0 || c >= kBN) return;
+#pragma unroll
+  for (int i = 0; i < kCols; ++i)
+    if (i == c) r[i] = __float_as_uint(__uint_as_float(r[i]) + delta);
+}
+
 template <typename T>
 __device__ __forceinline__ void store_row_chunk(T* dst, const float* v);  // 32 values
 
@@ -390,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = 64 * h;
             int u = t * p.bpt + r / p.b;
             if (u >= it.nblk) u = t * p.bpt;  // missing block: load a valid one, rows are not stored
-            const int y = it.blk(u) * p.b + (r % p.b);
+            const int y = qblock_start(p, it.blk(u)) + (r % p.b);  // rows past a short block: not stored
 #pragma unroll
             for (int c = 0; c < C::NCH; ++c)
               tma_load_3d(sQ + t * C::TILE + c * C::CH_STRIDE + h * 8192, &tm_q, &bars->q_full[t], c * C::BOX_X,
@@ -431,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const CUtensorMap* map;
             int y;
             if (new_rows) {
-              if (r0 < p.L_src) { map = &tm_k; y = r0; } else { map = &tm_ksel; y = r0 - p.L_src; }
+              if (r0 < p.L_srcp) { map = &tm_k; y = r0; } else { map = &tm_ksel; y = r0 - p.L_srcp; }
             } else {
               map = &tm_kcn; y = r0;
             }
@@ -458,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const CUtensorMap* map;
               int y;
               if (new_rows) {
-                if (r0 < p.L_src) { map = &tm_v; y = r0; } else { map = &tm_vsel; y = r0 - p.L_src; }
+                if (r0 < p.L_srcp) { map = &tm_v; y = r0; } else { map = &tm_vsel; y = r0 - p.L_srcp; }
               } else {
                 map = &tm_vcn; y = r0;
               }
@@ -643,14 +680,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = t * p.bpt + row / p.b;
         own = p.nsmask + ((size_t)it.bh * p.n_q + it.blk(u < it.nblk ? u : 0)) * p.ns_words;
       }
+      // short blocks: whether this head keeps the short last context block (the last of K_new)
+      const bool cs = p.ragged ? short_ctx_kept(p, it.bh) : false;
       for (int j = 0; j < it.nkv; ++j) {
         bool keep0 = true, keep1 = true;  // NS: this row keeps the K/V tile's first / second 64 keys
+        int len0 = 64, len1 = 64;         // NS: keys held by the tile's first / second 64 rows
         if constexpr (NS) {
           if (j >= p.npt) {
             const KeyTile kt = next_key_tile(p, it, cur, j);
             if (!tile_keeps(p, it, t, kt)) continue;  // no row of this tile keeps the K/V tile
             keep0 = has_block(own, kt.bk0);
             keep1 = p.b == 128 ? keep0 : has_block(own, kt.bk1);
+            if (p.ragged) {
+              const int l0 = new_block_len(p, kt.bk0, cs);
+              if (p.b == 128) {
+                len0 = min(l0, 64);
+                len1 = max(l0 - 64, 0);
+              } else {
+                len0 = l0;
+                len1 = kt.bk1 >= 0 ? new_block_len(p, kt.bk1, cs) : 0;
+              }
+            }
           }
         }
         if (!warp_wait(bars, &bars->s_full[t], s_cnt & 1, p.err)) { ok = false; break; }
@@ -674,15 +724,35 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 32; ++i)
                 r[32 * c + i] = (((mw >> i) & 1u) != 0u || 32 * c + i >= lim) ? kNegInf : r[32 * c + i];
             }
+            if (p.ragged) {  // a short block's pooled row weighs its own length
+              if (p.len_src_last < p.b) add_col_bias(r, j * kBN, p.n_src - 1, p.src_last_bias);
+              if (cs) add_col_bias(r, j * kBN, p.n_new - 1, p.ctx_last_bias);
+            }
           } else {
-            // exact blocks of the union: keep those in the row's own set
+            // exact blocks of the union: keep those in the row's own set (and, in a short
+            // block, only its keys)
 #pragma unroll
-            for (int i = 0; i < kCols; ++i) r[i] = (i < kCols / 2 ? keep0 : keep1) ? r[i] : kNegInf;
+            for (int i = 0; i < kCols; ++i)
+              r[i] = ((i < kCols / 2 ? keep0 : keep1) && (i & 63) < (i < kCols / 2 ? len0 : len1)) ? r[i] : kNegInf;
           }
-        } else if (j == it.nkv - 1 && it.last_valid < kBN) {  // ragged last K/V tile (uniform branch)
+        } else {
+          if (j == it.nkv - 1 && it.last_valid < kBN) {  // ragged last K/V tile (uniform branch)
 #pragma unroll
-          for (int i = 0; i < kCols; ++i)
-            if (i >= it.last_valid) r[i] = __float_as_uint(-INFINITY);
+            for (int i = 0; i < kCols; ++i)
+              if (i >= it.last_valid) r[i] = __float_as_uint(-INFINITY);
+          }
+          if (p.ragged) {
+            if (it.kind == 0) {
+              // exact path: the padding rows of the short source block and of a kept short
+              // context block (the last block of K_new)
+              mask_key_rows(r, j * kBN, p.L_src, p.L_srcp);
+              if (cs) mask_key_rows(r, j * kBN, p.L_new - (p.b - p.len_ctx_last), p.L_new);
+            } else {
+              // Taylor path: a short block's pooled row weighs its own length
+              if (p.len_src_last < p.b) add_col_bias(r, j * kBN, p.n_src - 1, p.src_last_bias);
+              if (cs) add_col_bias(r, j * kBN, p.n_new - 1, p.ctx_last_bias);
+            }
+          }
         }
         // row max of the raw scores: 8 independent chains of 3-input max
         float mc[8];
@@ -762,8 +832,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = 1.0f / l;
       if (!warp_wait(bars, &bars->o_done[t], (pv_cnt - 1) & 1, p.err)) { ok = false; break; }
       const int u = t * p.bpt + row / p.b;
-      const bool store = (u < it.nblk);
-      const size_t token = (size_t)it.blk(store ? u : 0) * p.b + (row % p.b);
+      const int qb = it.blk(u < it.nblk ? u : 0);
+      const bool store = (u < it.nblk) && (row % p.b) < qblock_len(p, qb);  // rows past a short block: none
+      const size_t token = (size_t)qblock_start(p, qb) + (row % p.b);
       T* dst = out + ((size_t)it.bh * p.N + token) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -812,6 +883,16 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, void* out, con
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   p.nsmask = w.nsmask;
   p.ns_words = pl.ns_words;
+  p.sel = w.sel;
+  p.k = pl.k;
+  p.n_src = pl.n_src;
+  p.n_ctx = pl.n_ctx;
+  p.L_srcp = pl.L_srcp;
+  p.len_src_last = pl.len_src_last;
+  p.len_ctx_last = pl.len_ctx_last;
+  p.ragged = pl.ragged;
+  p.src_last_bias = log2f((float)pl.len_src_last / (float)pl.b) / p.scale_log2;
+  p.ctx_last_bias = log2f((float)pl.len_ctx_last / (float)pl.b) / p.scale_log2;
   p.npt = (pl.n_new + kBN - 1) / kBN;
   p.bias_log2 = log2f((float)pl.b);
   if (NS && (pl.k_ns <= 0 || w.nsmask == nullptr)) return cudaErrorInvalidValue;

@@ -11,6 +11,9 @@
 // CTA moves one chunk of it with a pair of 1-D TMA bulk copies: global ->
 // shared (completion on an mbarrier), then shared -> global (bulk group).
 // Pure HBM traffic: 2 (K and V) x k x b x D elements read and written per head.
+// Every kept block takes b rows of K_sel / V_sel; when the last context block is
+// short (b does not divide L_ctx) and kept, its rows past its length are written
+// as zeros, so that the attention kernel's masked keys meet finite values.
 #include "isa_internal.h"
 #include "ptx.cuh"
 
@@ -33,18 +36,24 @@ __global__ void __launch_bounds__(32) gather_kernel(const char* __restrict__ k, 
   if (off >= blk_bytes) return;
   const uint32_t bytes = (uint32_t)((blk_bytes - off) < kChunk ? (blk_bytes - off) : kChunk);
   const int src_blk = w.sel[(size_t)bh * p.k + c];
+  const size_t valid = (size_t)(src_blk == p.n_ctx - 1 ? p.len_ctx_last : p.b) * row_bytes;
+  // bytes of this chunk that hold rows of the block (a multiple of the 128-byte-or-more row)
+  const uint32_t load = off >= valid ? 0u : (uint32_t)((valid - off) < bytes ? (valid - off) : bytes);
   const char* src = (which ? v : k) + ((size_t)bh * p.N + p.L_src + (size_t)src_blk * p.b) * row_bytes + off;
   char* dst = (which ? vsel : ksel) + ((size_t)bh * p.k + c) * blk_bytes + off;
 
-  mbar_init(&bar, 1);
-  mbar_fence_init();
-  mbar_arrive_expect_tx(&bar, bytes);
-  bulk_load(buf, src, bytes, &bar);
-  if (!mbar_wait(&bar, 0)) {
-    atomicOr(&w.ctrl[0], kErrGather);
-    // the load may still land; give it the same bound once more before leaving
-    mbar_wait(&bar, 0);
-    return;
+  for (uint32_t i = load; i < bytes; i += 16) *reinterpret_cast<uint4*>(buf + i) = make_uint4(0u, 0u, 0u, 0u);
+  if (load > 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+    mbar_arrive_expect_tx(&bar, load);
+    bulk_load(buf, src, load, &bar);
+    if (!mbar_wait(&bar, 0)) {
+      atomicOr(&w.ctrl[0], kErrGather);
+      // the load may still land; give it the same bound once more before leaving
+      mbar_wait(&bar, 0);
+      return;
+    }
   }
   fence_proxy_async_smem();
   bulk_store(dst, buf, bytes);

@@ -135,10 +135,13 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
   __syncthreads();
   auto issue = [&](int u, int s) {  // thread 0: the three blocks of unit u into stage s
     const int bh = u / p.n_q, blk = u - bh * p.n_q;
-    const size_t off = ((size_t)bh * p.N + (size_t)blk * BLK) * D;
+    // a block's rows are contiguous; the last block of the source or the context part may
+    // be short (its row count times D * E stays a multiple of 16 bytes)
+    const size_t off = ((size_t)bh * p.N + (size_t)block_start(p, blk)) * D;
+    const uint32_t bytes = (uint32_t)block_len(p, blk) * D * C::E;
     uint8_t* dst = smem + s * C::STAGE_BYTES;
-    mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-    for (int t = 0; t < 3; ++t) bulk_load(dst + t * C::TENSOR_BYTES, src[t] + off, C::TENSOR_BYTES, &full[s]);
+    mbar_arrive_expect_tx(&full[s], 3 * bytes);
+    for (int t = 0; t < 3; ++t) bulk_load(dst + t * C::TENSOR_BYTES, src[t] + off, bytes, &full[s]);
   };
   const int my_units = g < n_units ? (n_units - g + G - 1) / G : 0;
   int issued = 0;  // thread 0: units whose copies were started (unit i goes to stage i % STAGES)
@@ -156,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
       break;
     }
     const uint32_t* base = reinterpret_cast<const uint32_t*>(smem + s * C::STAGE_BYTES);
+    const int len = block_len(p, blk);  // rows of this block (BLK unless it is a short last block)
 #pragma unroll
     for (int t = 0; t < 3; ++t) {
       float acc[C::FPW];
@@ -163,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
       for (int f = 0; f < C::FPW; ++f) acc[f] = 0.f;
       const uint32_t* tb = base + t * (C::TENSOR_BYTES / 4);
 #pragma unroll 8
-      for (int r = rg; r < BLK; r += C::RG) add_word<T>(acc, tb[r * C::WPR + wd]);
+      for (int r = rg; r < len; r += C::RG) add_word<T>(acc, tb[r * C::WPR + wd]);
 #pragma unroll
       for (int f = 0; f < C::FPW; ++f) red[(t * C::RG + rg) * D + wd * C::FPW + f] = acc[f];
     }
@@ -173,14 +177,14 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
       issue(g + (i + C::STAGES) * G, s);
       ++issued;
     }
-    const float inv_b = 1.0f / (float)BLK;
+    const float inv_len = 1.0f / (float)len;
     for (int e = tid; e < 3 * D; e += kThreads) {
       const int t = e / D, c = e - t * D;
       float sum = 0.f;
 #pragma unroll
       for (int r = 0; r < C::RG; ++r) sum += red[(t * C::RG + r) * D + c];
       float* dst = (t == 0 ? w.qc : t == 1 ? w.kc : w.vc) + ((size_t)bh * p.n_q + blk) * D;
-      dst[c] = sum * inv_b;
+      dst[c] = sum * inv_len;
     }
     __syncthreads();  // `red` free for the next unit
   }

@@ -26,9 +26,12 @@ __global__ void __launch_bounds__(256) transpose_v_kernel(const float* __restric
     if (r < rows) {
       const float* src;
       if (pooled) src = static_cast<const float*>(w.vcn) + ((size_t)bh * p.n_new + r) * p.D;
-      else if (r < p.L_src) src = v + ((size_t)bh * p.N + r) * p.D;
-      else src = static_cast<const float*>(w.vsel) + ((size_t)bh * p.k * p.b + (r - p.L_src)) * p.D;
-      x = src[d0 + tx];
+      // K_new rows: the source part (read in place; rows L_src .. L_srcp - 1 of it are
+      // padding, masked by the attention kernel, and may lie past N), then the kept
+      // blocks, b rows each
+      else if (r < p.L_srcp) src = r < p.N ? v + ((size_t)bh * p.N + r) * p.D : nullptr;
+      else src = static_cast<const float*>(w.vsel) + ((size_t)bh * p.k * p.b + (r - p.L_srcp)) * p.D;
+      x = src ? src[d0 + tx] : 0.f;
     }
     tile[i][tx] = x;
   }

@@ -9,7 +9,7 @@
  * the source video and whose last L_ctx tokens are the context, one call runs:
  *
  *   1. pooling probe: Qc, Kc, Vc = means over blocks of b tokens;
- *      S_coarse = softmax(Qc Kc^T / sqrt(D)) over all n_q = N / b key blocks
+ *      S_coarse = softmax(Qc Kc^T / sqrt(D)) over all n_q key blocks
  *      (papernotes, Key design 1; paperlayer, section 2 "Pooling Attention");
  *   2. context pre-selection: score[c] = mean over the source query blocks of
  *      S_coarse[i, n_src + c]; keep the k = ceil(alpha_s * L_ctx / b) best
@@ -25,8 +25,11 @@
  *   5. both outputs written back in the original token order.
  *
  * Readings where the pages are silent (they are fixed here, and the CPU
- * oracle of the test suite follows the same ones): L_src and L_ctx are
- * multiples of b; k = ceil(alpha_s * n_ctx - 1e-4) and
+ * oracle of the test suite follows the same ones): the source tokens form
+ * n_src = ceil(L_src / b) blocks from token 0 and the context tokens
+ * n_ctx = ceil(L_ctx / b) blocks from token L_src, so the last block of
+ * either part may be short (its mean is over its own tokens, and in the
+ * Taylor path it weighs its own length instead of b); k = ceil(alpha_s * n_ctx - 1e-4) and
  * n_flat = floor(alpha_f * n_q + 1e-4), computed in double from the float
  * arguments; top-k and routing ties break by lower block index; kept blocks
  * enter K_new in ascending order after the source part.
@@ -34,7 +37,8 @@
  * Layout: q, k, v and out are row-major contiguous [B, H, N, D] with
  * N = L_src + L_ctx, in the element type given by isa_dtype (bfloat16 or
  * float32); out has the same type. Sizes supported: D in {64, 128}, b in
- * {64, 128}, N / b <= 2048; float32 only with D = 64.
+ * {64, 128}, any positive L_src and L_ctx with n_src + n_ctx <= 2048;
+ * float32 only with D = 64.
  *
  * Ownership: the caller owns every buffer passed in. The library never frees
  * caller memory and keeps no pointer after a call returns.
@@ -64,8 +68,8 @@ typedef enum { ISA_BF16 = 0, ISA_F32 = 1 } isa_dtype;
 enum {
   ISA_OK = 0,
   ISA_ERR_ARG = -1,         /* null or aliased pointer, non-positive size, ratio outside [0,1] or NaN */
-  ISA_ERR_SHAPE = -2,       /* L_src or L_ctx not a multiple of b */
-  ISA_ERR_UNSUPPORTED = -3, /* D, b, dtype or N / b outside the supported set */
+  ISA_ERR_SHAPE = -2,       /* reserved: lengths that b does not divide are accepted (short last blocks) */
+  ISA_ERR_UNSUPPORTED = -3, /* D, b, dtype or the block count outside the supported set */
   ISA_ERR_WORKSPACE = -4,   /* workspace null or smaller than isa_workspace_bytes() */
   ISA_ERR_CUDA = -5,        /* a CUDA runtime error; the message holds cudaGetErrorString() */
   ISA_ERR_TIMEOUT = -6      /* a kernel's bounded wait gave up (reported by isa_device_status) */
@@ -180,7 +184,7 @@ ISA_API int isa_set_stage_events(void* const* events, int n_events);
  *   q, k, v    device inputs [B, H, N, D] (as for isa_forward_ex)
  *   sel        device int32 [B, H, k] output: kept context blocks, ascending
  *   colscore   device float32 [B, H, N_ctx / b] output: context-block scores
- * Scratch (the block means of Q, K, V, 3 * B*H * (N/b) * D * 4 bytes, plus
+ * Scratch (the block means of Q, K, V, 3 * B*H * n_q * D * 4 bytes, plus
  * small partial sums, counters and control words, each part rounded up to 256
  * bytes) lives in a fixed 32 MiB device array inside the library, which
  * every GPU that loads the library holds until the process exits. Larger sizes

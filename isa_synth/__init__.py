@@ -140,19 +140,22 @@ def make_slice(w: Workload, seed: int, batch: int, head: int, attempt: int = 0,
     ``sigma_override`` (Q, K, V multipliers on the per-block sigma) lets tests
     build special cases, e.g. keys that are constant inside every block.
     """
-    if w.L_src % w.b or w.L_ctx % w.b:
-        raise ValueError("L_src and L_ctx must be multiples of b")
     rng = _slice_rng(seed, batch, head, attempt)
     N, D, b = w.N, w.D, w.b
-    n_q = N // b
+    # token -> block: source blocks of b tokens from 0, context blocks from L_src (the last
+    # block of either part is short when b does not divide its length)
+    n_src = -(-w.L_src // b)
+    tok = np.arange(N)
+    blk = np.where(tok < w.L_src, tok // b, n_src + (tok - w.L_src) // b)
+    n_q = int(blk[-1]) + 1
     sigma = rng.uniform(w.sigma_lo, w.sigma_hi, size=n_q)
-    blk_sigma = np.repeat(sigma, b)[:, None]
+    blk_sigma = sigma[blk][:, None]
     mult = sigma_override if sigma_override is not None else (1.0, 1.0, 1.0)
     outs = []
     for t in range(3):
         cent = rng.standard_normal((n_q, D))
         eps = rng.standard_normal((N, D))
-        x = np.repeat(cent, b, axis=0) + (mult[t] * blk_sigma) * eps
+        x = cent[blk] + (mult[t] * blk_sigma) * eps
         x[w.L_src:] *= w.s_ctx
         if w.dtype == "bf16":
             x = bf16_bits_to_f32(round_to_bf16_bits(x))

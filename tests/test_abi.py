@@ -75,7 +75,7 @@ def _fwd(L, q=FAKE, k=FAKE, v=FAKE, B=1, H=2, L_src=512, L_ctx=512, D=64, b=64, 
     (dict(B=0), -1), (dict(H=-1), -1), (dict(L_src=0), -1), (dict(L_ctx=-64), -1),
     (dict(a_s=float("nan")), -1), (dict(a_f=1.5), -1), (dict(a_s=-0.1), -1),
     (dict(D=96), -3), (dict(b=32), -3), (dict(dt=7), -3), (dict(dt=1, D=128), -3),
-    (dict(L_src=100), -2), (dict(L_ctx=96), -2),
+    (dict(L_src=100), -4), (dict(L_ctx=96), -4),   # short last blocks are accepted: no workspace here
     (dict(L_src=65536 * 2, L_ctx=64, b=64), -3),  # N / b above 2048
     (dict(B=70000, H=1), -3),
     (dict(), -4),                                  # no workspace
@@ -87,8 +87,6 @@ def test_argument_errors(L, kw, code):
 
 
 def test_plan_and_sizes_errors(L):
-    assert L.isa_workspace_bytes(1, 1, 100, 64, 64, 64, 0.5, 0) == 0
-    assert "multiples" in isa.last_error()
     with pytest.raises(isa.IsaError) as e:
         isa.plan(1, 1, 64, 64, 80, 64, 0.5, 0.5)
     assert e.value.code == -3
@@ -104,12 +102,13 @@ def test_workspace_grows_with_size(L):
 def test_launch_count(L):
     assert isa.launch_count(1, 40, 16384, 16384, 128, 128, 0.25, 0.6) == 4
     assert isa.launch_count(1, 40, 16384, 16384, 128, 128, 0.0, 0.6) == 3  # nothing to gather
-    assert isa.launch_count(1, 40, 100, 64, 128, 64, 0.25, 0.6) == 0
+    assert isa.launch_count(1, 40, 100, 64, 128, 64, 0.25, 0.6) == 4  # short last blocks: same launches
+    assert isa.launch_count(1, 40, 128, 64, 96, 64, 0.25, 0.6) == 0   # D = 96: invalid
 
 
 def test_host_entry_rejects_before_copying(L):
     assert L.isa_forward_host(None, FAKE, FAKE, 1, 1, 64, 64, 64, 64, 0.5, 0.5, 0, FAKE + 4096, None, None) == -1
-    assert L.isa_forward_host(FAKE, FAKE, FAKE, 1, 1, 64, 60, 64, 64, 0.5, 0.5, 0, FAKE + (1 << 30), None, None) == -2
+    assert L.isa_forward_host(FAKE, FAKE, FAKE, 1, 1, 64, 60, 96, 64, 0.5, 0.5, 0, FAKE + (1 << 30), None, None) == -3
 
 
 # ---------------------------------------------------------------- no-sparsity ratio alpha_ns
@@ -175,3 +174,16 @@ def test_pass_roofline():
     r = bench.pass_roofline(f, hb, ms=10.0, tflops=1000.0, gbs=5000.0)
     assert abs(r["t_roof_ms"] - (6.0 + 0.3)) < 1e-9
     assert abs(r["frac"] - 0.63) < 1e-12
+
+
+@pytest.mark.parametrize("L_src,L_ctx,b", [(100, 64, 64), (1000, 1100, 128), (65, 1, 64), (1, 200, 128)])
+def test_ragged_block_counts(L, L_src, L_ctx, b):
+    """Short last blocks: ceil(L_src / b) + ceil(L_ctx / b) blocks, k and n_flat as the ragged oracle's."""
+    from oracle import isa_oracle_ragged as R
+    bounds = R.block_bounds(L_src, L_ctx, b)
+    n_ctx = -(-L_ctx // b)
+    n_q, k, n_flat = isa.plan(1, 1, L_src, L_ctx, 64, b, 0.5, 0.5)
+    assert n_q == len(bounds)
+    assert k == O.kept_context_blocks(0.5, n_ctx) and n_flat == O.taylor_block_count(0.5, n_q)
+    # K_new takes b rows for every block, a short one padded
+    assert isa.workspace_bytes(1, 1, L_src, L_ctx, 64, b, 0.5) > 0
