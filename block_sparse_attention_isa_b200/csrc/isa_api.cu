@@ -187,6 +187,11 @@ inline cudaError_t mark(int i, cudaStream_t s) {
   return g_stage_events_on ? cudaEventRecord(g_stage_events[i], s) : cudaSuccess;
 }
 
+// The CTA-pair attention kernel runs the calls it supports with whole blocks; calls with a
+// short last block take the single-CTA kernel, which masks the padding rows of K_new and
+// weighs short pooled rows by their length.
+bool use_pair_kernel(const Plan& p) { return attention_pair_supported(p) && !p.ragged; }
+
 int run_forward(const void* q, const void* k, const void* v, const Plan& p, void* out, int32_t* dbg_sel,
                 int32_t* dbg_route, void* workspace, size_t workspace_bytes, cudaStream_t s) {
   const size_t need = workspace_layout(p, nullptr, nullptr);
@@ -211,7 +216,7 @@ int run_forward(const void* q, const void* k, const void* v, const Plan& p, void
     // takes the exact items only (its plan has no flat blocks; the route lists are unchanged)
     Plan pe = p;
     if (p.k_ns > 0) pe.n_flat = 0;
-    e = attention_pair_supported(pe) ? launch_attention_pair(q, k, v, out, pe, w, s, nullptr)
+    e = use_pair_kernel(pe) ? launch_attention_pair(q, k, v, out, pe, w, s, nullptr)
                                      : launch_attention(q, k, v, out, pe, w, s, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     if (p.k_ns > 0 && p.n_flat > 0 && (e = launch_attention_ns(q, k, v, out, p, w, s)) != cudaSuccess)

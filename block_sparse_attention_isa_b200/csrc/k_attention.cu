@@ -15,6 +15,12 @@
 //    gives the O(L_Q D) cost per query block that this reaches;
 //  * each output row is written at its original token position (each query
 //    block takes exactly one path, so there is nothing to merge).
+// When b does not divide L_src or L_ctx, the last block of either part is
+// short. K_new still takes b rows per block; the rows past a short block's keys
+// are masked. A short block's pooled row carries log2(len / b) on its exponent,
+// so that in the Taylor path it weighs its own length (the weight no longer
+// cancels for it). Query rows are addressed by block start, and only a block's
+// own rows are stored. Such calls are run by this kernel, not the CTA-pair one.
 //
 // Design for sm_100a (prior art on the pages is Triton / TileLang on Hopper):
 //  * one CTA per SM (persistent), 12 warps: warp 0 issues TMA loads, warp 1

@@ -598,9 +598,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-// Calls with a short last block (b not dividing L_src or L_ctx) take the single-CTA kernel,
-// which masks the padding rows of K_new and weighs short pooled rows by their length.
-bool attention_pair_supported(const Plan& p) { return p.dt == 0 && p.D == kD && !p.ragged; }
+bool attention_pair_supported(const Plan& p) { return p.dt == 0 && p.D == kD; }
 
 cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, void* out, const Plan& pl,
                                   const Work& w, cudaStream_t s, int* n_ctas) {

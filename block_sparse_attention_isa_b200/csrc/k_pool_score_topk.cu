@@ -7,14 +7,17 @@
 // papernotes.org notes, Key design 1 (Context Pre-Selection), and the
 // paperlayer.ai summary, section 2 (Pooling Attention) and section 3
 // (Pre-Selection):
-//   Qc, Kc, Vc = means over blocks of b tokens,
+//   Qc, Kc, Vc = means over blocks of b tokens (source blocks from token 0,
+//     context blocks from token L_src; the last block of either part may be
+//     short, and its mean is over its own tokens),
 //   S_coarse[i, :] = softmax_j(Qc_i . Kc_j / sqrt(D)) for source blocks i,
 //   score[c] = mean_i S_coarse[i, n_src + c],
 //   sel = the k largest scores (ties by lower index), stored ascending.
 //
 // One persistent cooperative launch, one CTA per SM, 256 threads:
 //  * phase 1 (HBM-bound): pooling units (head, block) are dealt round-robin to
-//    the CTAs; each unit's Q, K and V blocks (b contiguous rows each) arrive in
+//    the CTAs; each unit's Q, K and V blocks (b contiguous rows each, fewer in a
+//    short last block) arrive in
 //    a ring of shared-memory stages by 1-D TMA bulk copies, so several units
 //    are in flight per SM while the previous one is reduced (fp32 sums, 4-byte
 //    words, conflict-free shared-memory reads);
