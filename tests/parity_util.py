@@ -1,5 +1,4 @@
 """Helpers shared by the GPU parity tests: input drawing with near-tie rejection, GPU runs, comparisons."""
-import math
 
 import numpy as np
 

@@ -5,8 +5,6 @@ before touching CUDA, or only computes sizes. Fake device addresses are only
 ever passed together with a missing or undersized workspace, which the library
 rejects before any CUDA call.
 """
-import ctypes
-import math
 import os
 import re
 import subprocess

@@ -8,7 +8,6 @@ isa_forward_ex, which uses a caller workspace: the kept context blocks exactly,
 the context scores within the tolerance of the stage tests. This file is
 collected last so that a failure here cannot stop the rest of a -x run.
 """
-import ctypes
 
 import numpy as np
 import pytest
