@@ -6,10 +6,16 @@ A step is one ISA forward call over the headline workload (B=1, H=40, D=128,
 L_src = L_ctx = 16384, b = 128, alpha_s = 0.25, alpha_f = 0.6: the 32K-token
 case), inputs resident in HBM. `value` is the effective throughput in TFLOP/s
 (FLOPs the pass executes: coarse scores, routing, exact and Taylor attention)
-over all ranks; `ms_per_step` is the max over ranks. Under torchrun each rank
-runs its own replica of the workload (independent batches: weak scaling, no
-collective on the data path; NCCL only for the barrier and the max of the
-timings).
+over all ranks; `ms_per_step` is the max over ranks.
+
+Under torchrun the (batch, head) slices are the units that ranks share:
+* `--scaling weak` (default): rank r computes batch element r of a global
+  batch of N elements (its own draw of the workload's shape), so per-GPU work
+  is fixed; no collective on the data path (NCCL only for the barrier and the
+  max of the timings);
+* `--scaling strong`: the workload's B*H slices are split into contiguous
+  ranges over the ranks; with `--gather` the timed step also all-gathers O
+  over NCCL so that every rank holds the whole output.
 
 `--impl reference` times the CPU oracle (float64 numpy) as it stands on the
 host cores over a bounded sample of the same workload (one head per step).
@@ -171,12 +177,29 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- arms
 
-def workload_inputs(w, seed=0, full=None):
-    """Q, K, V of workload w; with `full` (w = full with fewer heads) its first heads, same draws."""
+def workload_inputs(w, seed=0, full=None, batch=0):
+    """Q, K, V of workload w; with `full` (w = full with fewer heads) its first heads, same draws.
+
+    `batch` > 0 draws batch element `batch` instead (B = 1; the weak-scaling unit of rank `batch`)."""
+    if batch:
+        q = np.zeros((1, w.H, w.N, w.D), np.float32)
+        k, v = np.zeros_like(q), np.zeros_like(q)
+        for h in range(w.H):
+            q[0, h], k[0, h], v[0, h] = isa_synth.make_slice(w, seed, batch, h, 0)
+        return q, k, v
     att = isa_synth.attempts_for(full or w, seed)
     if att is not None and full is not None:
         att = att[:, :w.H]
     return isa_synth.make_inputs(w, seed, att)
+
+
+def roofline_peak(peaks: dict, timed_s: float) -> tuple:
+    """(peak TFLOP/s, kind) for a kernel timed over `timed_s` seconds: the burst GEMM figure
+    when the timed region is shorter than a second (below the power cap's reaction time),
+    else the sustained one."""
+    if timed_s < 1.0 or "bf16_tflops_sustained" not in peaks:
+        return peaks["bf16_tflops"], "burst"
+    return peaks["bf16_tflops_sustained"], "sustained"
 
 
 def bf16_bits(x):
@@ -265,6 +288,7 @@ def run_ours(args, w):
 
     import block_sparse_attention_isa_b200 as isa
     from block_sparse_attention_isa_b200 import build as isa_build
+    from block_sparse_attention_isa_b200 import sharding
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -276,19 +300,29 @@ def run_ours(args, w):
     isa_build.build()
     dev = torch.device("cuda", local)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    strong = args.scaling == "strong" and world > 1
 
-    q, k, v = workload_inputs(w, full=getattr(args, "full_workload", None))
+    # weak scaling: rank r computes its own batch element r; strong: rank r computes its range of
+    # the workload's slices (every rank draws the same whole workload and uses its range)
+    q, k, v = workload_inputs(w, full=getattr(args, "full_workload", None), batch=0 if strong else rank)
     tq, tk, tv = (torch.from_numpy(x).to(dev, dt) for x in (q, k, v))
+    s0, s1 = sharding.slice_range(rank, world, w.B * w.H) if strong else (0, w.B * w.H)
+    wr = w.with_(B=1, H=s1 - s0) if strong else w  # this rank's call
+    if strong:
+        tq, tk, tv = (t.reshape(w.B * w.H, w.N, w.D)[s0:s1].unsqueeze(0).contiguous() for t in (tq, tk, tv))
     out = torch.empty_like(tq)
     a_ns = args.alpha_ns
-    ws = torch.empty(isa.workspace_bytes(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s,
-                                         isa.ISA_BF16 if w.dtype == "bf16" else isa.ISA_F32, alpha_ns=a_ns),
+    dtc = isa.ISA_BF16 if w.dtype == "bf16" else isa.ISA_F32
+    ws = torch.empty(isa.workspace_bytes(wr.B, wr.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, dtc, alpha_ns=a_ns),
                      dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    gather = strong and args.gather
 
     def step():
         isa.forward_into(tq, tk, tv, out, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, workspace=ws, stream=stream,
                          alpha_ns=a_ns)
+        if gather:
+            sharding.gather_output(out.reshape(s1 - s0, w.N, w.D), w.B, w.H)
 
     for _ in range(args.warmup):
         step()
@@ -324,16 +358,21 @@ def run_ours(args, w):
     max_ms = reduce_max(ms, dist)
     stage_ms = {name: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)) / args.steps
                 for i, name in enumerate(isa.STAGES)}
-    f = flops_per_call(w, a_ns)
-    hb = hbm_bytes_per_call(w)
+    f = flops_per_call(wr, a_ns)          # this rank's call
+    f_job = flops_per_call(w, a_ns)       # one unit of the whole job (the workload)
+    hb = hbm_bytes_per_call(wr)
     peaks, peaks_kind = load_peaks()
     attn_tflops = (f["exact"] + f["taylor"]) / (stage_ms["attention"] * 1e-3) / 1e12
+    peak, peak_which = roofline_peak(peaks, args.steps * ms * 1e-3)
     peak_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     pool_gbs = hb["pool"] / (stage_ms["pool_score_topk"] * 1e-3) / 1e9
     gather_gbs = hb["gather"] / max(stage_ms["gather"] * 1e-3, 1e-12) / 1e9
+    # clock-normalised: the attention time scaled to the maximum SM clock (a power-capped run
+    # that ran at a lower median clock reads as the same kernel at full clock)
+    clock_ratio = (clk["sm_mhz"] / clk["sm_max_mhz"]) if clk.get("sm_mhz") and clk.get("sm_max_mhz") else None
     traffic = None
     prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof) and not a_ns:  # (the counters cover the plain path's attention kernel only)
+    if os.path.exists(prof) and not a_ns and not strong:  # (counters of the plain path's attention kernel only)
         with open(prof) as fh:
             ent = json.load(fh).get(w.name, {})
         # the counters hold only for the kernel source they were taken on
@@ -342,20 +381,20 @@ def run_ours(args, w):
 
     # end to end through the host-buffer entry point (pinned host memory, copies inside the timed region)
     e2e = None
-    # (the host-buffer entry point has no alpha_ns argument: no end-to-end figure for that variant)
-    if not args.no_e2e and not a_ns and (rank == 0 or world > 1):
+    if not args.no_e2e and (rank == 0 or world > 1):
         hq, hk, hv = (t.cpu().pin_memory() for t in (tq, tk, tv))
         hout = torch.empty_like(hq).pin_memory()
         n_e2e = max(1, min(args.steps, 5))
-        isa.forward_host(hq, hk, hv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, out=hout)
+        isa.forward_host(hq, hk, hv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, out=hout, alpha_ns=a_ns)
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         for _ in range(n_e2e):
-            isa.forward_host(hq, hk, hv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, out=hout)
+            isa.forward_host(hq, hk, hv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, out=hout, alpha_ns=a_ns)
         e2e_ms = (time.perf_counter() - t0) / n_e2e * 1e3
         e2e_ms = reduce_max(e2e_ms, dist)
         nbytes = hq.numel() * hq.element_size()
-        e2e = {"value": aggregate(f["total"], e2e_ms, world), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e_val = f_job["total"] / (e2e_ms * 1e-3) / 1e12 if strong else aggregate(f["total"], e2e_ms, world)
+        e2e = {"value": e2e_val, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
 
     cpu = None
@@ -365,25 +404,39 @@ def run_ours(args, w):
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
                "sample": f"{done} of {w.B * w.H} heads of the same workload, {secs:.1f} s of CPU time"}
 
-    launches = isa.launch_count(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, w.alpha_f,
-                                isa.ISA_BF16 if w.dtype == "bf16" else isa.ISA_F32, alpha_ns=a_ns)
+    launches = isa.launch_count(wr.B, wr.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, w.alpha_f, dtc, alpha_ns=a_ns)
     if rank == 0:
+        value = f_job["total"] / (max_ms * 1e-3) / 1e12 if strong else aggregate(f["total"], max_ms, world)
+        parallelism = (f"heads split over {world} ranks" + (" + NCCL all-gather of O" if gather else "")
+                       if strong else (f"dp{world} (rank r computes batch element r)" if world > 1 else "single GPU"))
+        exact_t = f["exact"] / (stage_ms["attention"] * 1e-3) / 1e12
         line = {
-            "metric": METRIC, "value": aggregate(f["total"], max_ms, world), "unit": "TFLOP/s", "n_gpus": world,
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
-            "data": "synthetic",
+            "scaling": "strong" if strong else "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": workload_label(args, w), "B": w.B, "H": w.H, "N": w.N, "D": w.D, "b": w.b,
-                       "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "alpha_ns": a_ns, "global_batch": w.B * world,
-                       "seq_len": w.N, "parallelism": f"replicas x{world}",
+                       "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "alpha_ns": a_ns,
+                       "global_batch": w.B if strong else w.B * world, "seq_len": w.N, "parallelism": parallelism,
                        "l2": "inputs larger than L2 (Q, K, V = %.2f GB per step)" % (3 * tq.numel() * tq.element_size() / 1e9)},
             "roofline": {"bound": "tensor", "kernel": "attention (exact + Taylor paths)", "achieved": attn_tflops,
-                         "peak": peak_sust, "unit": "TFLOP/s", "frac": attn_tflops / peak_sust,
-                         "peak_kind": f"{peaks_kind} bf16 sustained",
+                         "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                         "peak_kind": f"{peaks_kind} bf16 {peak_which} (timed region {args.steps * ms / 1e3:.2f} s)",
                          "frac_of_burst": attn_tflops / peaks["bf16_tflops"],
-                         "frac_of_nominal": attn_tflops / NOMINAL["bf16_tflops"], "traffic": traffic},
-            "pass_roofline": {"measured": pass_roofline(f, hb, max_ms, peak_sust, peaks["hbm_gbs"]),
-                              "nominal": pass_roofline(f, hb, max_ms, NOMINAL["bf16_tflops"], NOMINAL["hbm_gbs"])},
+                         "frac_of_sustained": attn_tflops / peak_sust,
+                         "frac_of_nominal": attn_tflops / NOMINAL["bf16_tflops"],
+                         # the exact path's FLOPs over the whole attention time (Taylor items included):
+                         # a lower bound on the exact path's own fraction
+                         "exact_path_frac_lower_bound": exact_t / peak,
+                         "flops_share": {"exact": f["exact"] / (f["exact"] + f["taylor"]),
+                                         "taylor": f["taylor"] / (f["exact"] + f["taylor"])},
+                         "traffic": traffic},
+            "clock_normalised": None if clock_ratio is None else {
+                "sm_mhz_median": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
+                "attention_ms_at_max_clock": stage_ms["attention"] * clock_ratio,
+                "frac_at_max_clock": attn_tflops / clock_ratio / peak},
+            "pass_roofline": {"measured": pass_roofline(f, hb, ms, peak, peaks["hbm_gbs"]),
+                              "nominal": pass_roofline(f, hb, ms, NOMINAL["bf16_tflops"], NOMINAL["hbm_gbs"])},
             "stages_ms": stage_ms,
             "hbm_stages": {"pool_score_topk_gbs": pool_gbs, "gather_gbs": gather_gbs,
                            "pool_frac": pool_gbs / peaks["hbm_gbs"], "gather_frac": gather_gbs / peaks["hbm_gbs"],
@@ -414,6 +467,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--alpha-ns", type=float, default=0.0,
                     help="no-sparsity ratio: exact key blocks inside the Taylor path (bf16 only; 0 = plain path)")
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
+                    help="N > 1: weak = one batch element per rank; strong = the workload's heads split over ranks")
+    ap.add_argument("--gather", action="store_true", help="strong scaling: all-gather O over NCCL in every step")
     ap.add_argument("--heads", type=int, default=0,
                     help="run only the first H heads of the workload (small profiling captures; not a bench line)")
     args = ap.parse_args()

@@ -25,6 +25,8 @@ __all__ = [
     "forward",
     "forward_into",
     "forward_host",
+    "select_context_noalloc",
+    "select_context_noalloc_status",
     "device_status",
     "debug_pooled",
     "selftest_wait_timeout",
@@ -61,6 +63,8 @@ EXPORTS = (
     "isa_selftest_exp2",
     "isa_set_stage_events",
     "isa_select_context_noalloc",
+    "isa_select_context_noalloc_status",
+    "isa_forward_host_ns",
     "isa_plan_ns",
     "isa_workspace_bytes_ns",
     "isa_forward_ns",
@@ -120,6 +124,10 @@ def lib() -> ctypes.CDLL:
     L.isa_set_stage_events.restype = c_int
     L.isa_select_context_noalloc.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_int, vp, vp, vp]
     L.isa_select_context_noalloc.restype = c_int
+    L.isa_select_context_noalloc_status.argtypes = [vp]
+    L.isa_select_context_noalloc_status.restype = c_int
+    L.isa_forward_host_ns.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_float, c_float, c_int, vp, vp, vp]
+    L.isa_forward_host_ns.restype = c_int
     L.isa_plan_ns.argtypes = [c_int] * 6 + [c_float, c_float, c_float, i32p, i32p, i32p, i32p]
     L.isa_plan_ns.restype = c_int
     L.isa_workspace_bytes_ns.argtypes = [c_int] * 6 + [c_float, c_float, c_int]
@@ -317,11 +325,36 @@ def debug_pooled(B, H, L_src, L_ctx, D, b, alpha_s, dtype=ISA_BF16, workspace=No
     return res
 
 
+def select_context_noalloc(q, k, v, L_src: int, L_ctx: int, b: int, alpha_s: float, sel, colscore, stream=None):
+    """Stages 1-2 through the allocation-free entry point (scratch in the library's fixed array).
+
+    Enqueues only; call ``select_context_noalloc_status`` before the next call to learn whether
+    the kernel's bounded waits gave up."""
+    torch = _torch()
+    B, H, N, D = q.shape
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    s = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    _check(lib().isa_select_context_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, L_src, L_ctx, D, b,
+                                            alpha_s, _dtype_code(q), sel.data_ptr(), colscore.data_ptr(), s))
+
+
+def select_context_noalloc_status(stream=None):
+    """Synchronise and raise IsaError(ISA_ERR_TIMEOUT) if the last allocation-free call's wait gave up."""
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    s = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    _check(lib().isa_select_context_noalloc_status(s))
+
+
 def forward_host(q, k, v, L_src: int, L_ctx: int, b: int, alpha_s: float, alpha_f: float, out=None,
-                 dbg_sel=None, dbg_route=None, dtype: Optional[int] = None):
+                 dbg_sel=None, dbg_route=None, dtype: Optional[int] = None, alpha_ns: float = 0.0):
     """The pass on HOST buffers (numpy arrays or CPU tensors, pinned or not): copies in, runs, copies out.
 
     For bfloat16, pass uint16 numpy arrays holding the bit patterns, or bfloat16 CPU tensors.
+    With ``alpha_ns`` > 0 the Taylor query blocks keep their k_ns best K_new blocks exact
+    (isa_forward_host_ns).
     """
     import numpy as np
 
@@ -344,6 +377,10 @@ def forward_host(q, k, v, L_src: int, L_ctx: int, b: int, alpha_s: float, alpha_
             dtype = _dtype_code(q)
     if out is None:
         out = np.empty_like(q) if isinstance(q, np.ndarray) else _torch().empty_like(q)
+    if alpha_ns:
+        _check(lib().isa_forward_host_ns(ptr(q), ptr(k), ptr(v), B, H, L_src, L_ctx, D, b, alpha_s, alpha_f,
+                                         alpha_ns, dtype, ptr(out), ptr(dbg_sel), ptr(dbg_route)))
+        return out
     _check(lib().isa_forward_host(ptr(q), ptr(k), ptr(v), B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dtype,
                                   ptr(out), ptr(dbg_sel), ptr(dbg_route)))
     return out

@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/isa.h"
 #include "isa_internal.h"
@@ -242,6 +243,22 @@ int check_io(const void* q, const void* k, const void* v, const void* out, const
   return ISA_OK;
 }
 
+// Device buffers are read and written by bulk and tensor copies, which need 16-byte
+// aligned addresses: a misaligned pointer is an argument error, not a launch.
+int check_aligned(const void* q, const void* k, const void* v, const void* out) {
+  const void* ptrs[4] = {q, k, v, out};
+  const char* names[4] = {"q", "k", "v", "out"};
+  for (int i = 0; i < 4; ++i)
+    if (ptrs[i] && (reinterpret_cast<uintptr_t>(ptrs[i]) & 15))
+      return fail(ISA_ERR_ARG, "%s must be 16-byte aligned (device address %p)", names[i], ptrs[i]);
+  return ISA_OK;
+}
+
+int check_device_io(const void* q, const void* k, const void* v, const void* out, const Plan& p) {
+  const int rc = check_io(q, k, v, out, p);
+  return rc != ISA_OK ? rc : check_aligned(q, k, v, out);
+}
+
 int read_status(void* workspace, cudaStream_t s) {
   cudaError_t e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "synchronising the stream");
@@ -253,6 +270,88 @@ int read_status(void* workspace, cudaStream_t s) {
     return fail(ISA_ERR_TIMEOUT, "a kernel wait timed out (error word 0x%x)", word);
   }
   return ISA_OK;
+}
+
+// Device buffers of the host-buffer entry points come from a stream-ordered memory pool that
+// belongs to this library (one per device, created on first use), not from the device's default
+// pool: its release threshold is raised so that repeated calls reuse the memory instead of
+// returning it to the driver, and the caller's pools keep whatever settings they had.
+int host_pool(cudaMemPool_t* out) {
+  static cudaMemPool_t pools[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(ISA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool;
+    if ((e = cudaMemPoolCreate(&pool, &props)) != cudaSuccess) return cuda_fail(e, "creating the library's memory pool");
+    uint64_t thr = UINT64_MAX;
+    if ((e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr)) != cudaSuccess)
+      return cuda_fail(e, "configuring the library's memory pool");
+    pools[dev] = pool;
+  }
+  *out = pools[dev];
+  return ISA_OK;
+}
+
+// The pass on host buffers: copies in, runs the pass (alpha_ns as for isa_forward_ns), copies
+// out and synchronises.
+int host_forward(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
+                 float alpha_s, float alpha_f, float alpha_ns, isa_dtype dt, void* out, int32_t* dbg_sel,
+                 int32_t* dbg_route) {
+  Plan p;
+  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p, alpha_ns);
+  if (rc != ISA_OK) return rc;
+  if ((rc = check_io(q, k, v, out, p)) != ISA_OK) return rc;
+  const size_t io = align256((size_t)p.BH * p.N * p.D * p.elem);
+  const size_t ws_bytes = workspace_layout(p, nullptr, nullptr);
+  const size_t sel_b = align256(sizeof(int32_t) * (size_t)p.BH * (p.k > 0 ? p.k : 1));
+  const size_t route_b = align256(sizeof(int32_t) * (size_t)p.BH * p.n_q);
+  const size_t total = 4 * io + ws_bytes + sel_b + route_b;
+  cudaStream_t s = 0;
+  cudaMemPool_t pool;
+  if ((rc = host_pool(&pool)) != ISA_OK) return rc;
+  char* dev_buf = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&dev_buf), total, pool, s);
+  if (e != cudaSuccess) return cuda_fail(e, "allocating device buffers");
+  char* dq = dev_buf;
+  char* dk = dq + io;
+  char* dv = dk + io;
+  char* dout = dv + io;
+  char* dws = dout + io;
+  int32_t* dsel = reinterpret_cast<int32_t*>(dws + ws_bytes);
+  int32_t* droute = reinterpret_cast<int32_t*>(dws + ws_bytes + sel_b);
+  const size_t bytes = (size_t)p.BH * p.N * p.D * p.elem;
+  rc = ISA_OK;
+  if ((e = cudaMemcpyAsync(dq, q, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dk, k, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dv, v, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+    rc = cuda_fail(e, "copying inputs to the device");
+  if (rc == ISA_OK)
+    rc = run_forward(dq, dk, dv, p, dout, dbg_sel ? dsel : nullptr, dbg_route ? droute : nullptr, dws, ws_bytes, s);
+  if (rc == ISA_OK && (e = cudaMemcpyAsync(out, dout, bytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    rc = cuda_fail(e, "copying the output to the host");
+  if (rc == ISA_OK && dbg_sel && p.k > 0 &&
+      (e = cudaMemcpyAsync(dbg_sel, dsel, sizeof(int32_t) * (size_t)p.BH * p.k, cudaMemcpyDeviceToHost, s)) !=
+          cudaSuccess)
+    rc = cuda_fail(e, "copying dbg_sel to the host");
+  if (rc == ISA_OK && dbg_route &&
+      (e = cudaMemcpyAsync(dbg_route, droute, sizeof(int32_t) * (size_t)p.BH * p.n_q, cudaMemcpyDeviceToHost, s)) !=
+          cudaSuccess)
+    rc = cuda_fail(e, "copying dbg_route to the host");
+  const int st = read_status(dws, s);
+  if (rc == ISA_OK) rc = st;
+  cudaFreeAsync(dev_buf, s);
+  e = cudaStreamSynchronize(s);
+  if (rc == ISA_OK && e != cudaSuccess) rc = cuda_fail(e, "releasing device buffers");
+  return rc;
 }
 
 }  // namespace
@@ -319,7 +418,7 @@ int isa_forward_ns(const void* q, const void* k, const void* v, int B, int H, in
   Plan p;
   int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p, alpha_ns);
   if (rc != ISA_OK) return rc;
-  if ((rc = check_io(q, k, v, out, p)) != ISA_OK) return rc;
+  if ((rc = check_device_io(q, k, v, out, p)) != ISA_OK) return rc;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   rc = run_forward(q, k, v, p, out, dbg_sel, dbg_route, workspace, workspace_bytes, s);
   if (rc != ISA_OK || !dbg_ns || p.k_ns == 0) return rc;
@@ -336,7 +435,7 @@ int isa_forward_ex(const void* q, const void* k, const void* v, int B, int H, in
   Plan p;
   int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p);
   if (rc != ISA_OK) return rc;
-  if ((rc = check_io(q, k, v, out, p)) != ISA_OK) return rc;
+  if ((rc = check_device_io(q, k, v, out, p)) != ISA_OK) return rc;
   return run_forward(q, k, v, p, out, dbg_sel, dbg_route, workspace, workspace_bytes,
                      static_cast<cudaStream_t>(stream));
 }
@@ -346,7 +445,7 @@ int isa_forward(const void* q, const void* k, const void* v, int B, int H, int L
   Plan p;
   int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, ISA_BF16, &p);
   if (rc != ISA_OK) return rc;
-  if ((rc = check_io(q, k, v, out, p)) != ISA_OK) return rc;
+  if ((rc = check_device_io(q, k, v, out, p)) != ISA_OK) return rc;
   const size_t ws_bytes = workspace_layout(p, nullptr, nullptr);
   void* ws = nullptr;
   cudaStream_t s = 0;
@@ -363,58 +462,13 @@ int isa_forward(const void* q, const void* k, const void* v, int B, int H, int L
 
 int isa_forward_host(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
                      float alpha_s, float alpha_f, isa_dtype dt, void* out, int32_t* dbg_sel, int32_t* dbg_route) {
-  Plan p;
-  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p);
-  if (rc != ISA_OK) return rc;
-  if ((rc = check_io(q, k, v, out, p)) != ISA_OK) return rc;
-  const size_t io = align256((size_t)p.BH * p.N * p.D * p.elem);
-  const size_t ws_bytes = workspace_layout(p, nullptr, nullptr);
-  const size_t sel_b = align256(sizeof(int32_t) * (size_t)p.BH * (p.k > 0 ? p.k : 1));
-  const size_t route_b = align256(sizeof(int32_t) * (size_t)p.BH * p.n_q);
-  const size_t total = 4 * io + ws_bytes + sel_b + route_b;
-  cudaStream_t s = 0;
-  // keep freed blocks in the stream-ordered pool so that repeated calls do not
-  // go back to the driver for memory
-  int dev = 0;
-  cudaMemPool_t pool;
-  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
-    uint64_t thr = UINT64_MAX;
-    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
-  }
-  char* dev_buf = nullptr;
-  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&dev_buf), total, s);
-  if (e != cudaSuccess) return cuda_fail(e, "allocating device buffers");
-  char* dq = dev_buf;
-  char* dk = dq + io;
-  char* dv = dk + io;
-  char* dout = dv + io;
-  char* dws = dout + io;
-  int32_t* dsel = reinterpret_cast<int32_t*>(dws + ws_bytes);
-  int32_t* droute = reinterpret_cast<int32_t*>(dws + ws_bytes + sel_b);
-  const size_t bytes = (size_t)p.BH * p.N * p.D * p.elem;
-  rc = ISA_OK;
-  if ((e = cudaMemcpyAsync(dq, q, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(dk, k, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(dv, v, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
-    rc = cuda_fail(e, "copying inputs to the device");
-  if (rc == ISA_OK)
-    rc = run_forward(dq, dk, dv, p, dout, dbg_sel ? dsel : nullptr, dbg_route ? droute : nullptr, dws, ws_bytes, s);
-  if (rc == ISA_OK && (e = cudaMemcpyAsync(out, dout, bytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
-    rc = cuda_fail(e, "copying the output to the host");
-  if (rc == ISA_OK && dbg_sel && p.k > 0 &&
-      (e = cudaMemcpyAsync(dbg_sel, dsel, sizeof(int32_t) * (size_t)p.BH * p.k, cudaMemcpyDeviceToHost, s)) !=
-          cudaSuccess)
-    rc = cuda_fail(e, "copying dbg_sel to the host");
-  if (rc == ISA_OK && dbg_route &&
-      (e = cudaMemcpyAsync(dbg_route, droute, sizeof(int32_t) * (size_t)p.BH * p.n_q, cudaMemcpyDeviceToHost, s)) !=
-          cudaSuccess)
-    rc = cuda_fail(e, "copying dbg_route to the host");
-  const int st = read_status(dws, s);
-  if (rc == ISA_OK) rc = st;
-  cudaFreeAsync(dev_buf, s);
-  e = cudaStreamSynchronize(s);
-  if (rc == ISA_OK && e != cudaSuccess) rc = cuda_fail(e, "releasing device buffers");
-  return rc;
+  return host_forward(q, k, v, B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, 0.0f, dt, out, dbg_sel, dbg_route);
+}
+
+int isa_forward_host_ns(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D,
+                        int b, float alpha_s, float alpha_f, float alpha_ns, isa_dtype dt, void* out,
+                        int32_t* dbg_sel, int32_t* dbg_route) {
+  return host_forward(q, k, v, B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, alpha_ns, dt, out, dbg_sel, dbg_route);
 }
 
 int isa_selftest_wait_timeout(void* workspace, int timeout_ms, void* stream) {

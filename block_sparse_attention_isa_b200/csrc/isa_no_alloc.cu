@@ -14,7 +14,11 @@
 // loads this library holds that array until the process exits. Host code must
 // not pass the symbol itself to a kernel (on the host it names a host-side
 // stand-in); the device address is looked up once per device with
-// cudaGetSymbolAddress and cached.
+// cudaGetSymbolAddress and cached. The cache does not survive cudaDeviceReset.
+//
+// The kernel's bounded waits report a give-up in the error word at the start of
+// the array; isa_select_context_noalloc_status synchronises the stream and reads
+// and clears that word, so that a call that timed out is not taken for a good one.
 #include <mutex>
 
 #include "../../include/isa.h"
@@ -31,6 +35,17 @@ void* g_scratch_addr[kMaxDevices] = {};
 std::mutex g_scratch_mutex;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Device address of g_scratch on the current device, or NULL when no call has looked it up yet.
+int scratch_address_if_known(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return set_error(ISA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  *out = g_scratch_addr[dev];
+  return ISA_OK;
+}
 
 // Device address of g_scratch on the current device (looked up on first use).
 int scratch_address(void** out) {
@@ -63,6 +78,16 @@ extern "C" int isa_select_context_noalloc(const void* q, const void* k, const vo
   if (rc != ISA_OK) return rc;
   if (!q || !k || !v) return set_error(ISA_ERR_ARG, "q, k and v must not be NULL");
   if (!sel || !colscore) return set_error(ISA_ERR_ARG, "sel and colscore must not be NULL");
+  {
+    // the pooling kernel reads the inputs with bulk copies, which need 16-byte aligned addresses
+    const void* ptrs[3] = {q, k, v};
+    const char* names[3] = {"q", "k", "v"};
+    for (int i = 0; i < 3; ++i)
+      if (reinterpret_cast<uintptr_t>(ptrs[i]) & 15)
+        return set_error(ISA_ERR_ARG, "%s must be 16-byte aligned (device address %p)", names[i], ptrs[i]);
+    if ((reinterpret_cast<uintptr_t>(sel) & 3) || (reinterpret_cast<uintptr_t>(colscore) & 3))
+      return set_error(ISA_ERR_ARG, "sel and colscore must be 4-byte aligned");
+  }
   const size_t BH = (size_t)p.BH;
   const size_t ctrl_bytes = align256(sizeof(uint32_t) * kCtrlWords);
   const size_t ctr_bytes = align256(sizeof(uint32_t) * BH);
@@ -93,5 +118,24 @@ extern "C" int isa_select_context_noalloc(const void* q, const void* k, const vo
   if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "clearing the scratch counters: %s", cudaGetErrorString(e));
   e = launch_pool_score_topk(q, k, v, p, w, s);
   if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "pool/score/top-k launch: %s", cudaGetErrorString(e));
+  return ISA_OK;
+}
+
+extern "C" int isa_select_context_noalloc_status(void* stream) {
+  void* base = nullptr;
+  int rc = scratch_address_if_known(&base);
+  if (rc != ISA_OK) return rc;
+  if (!base) return ISA_OK;  // no call has run on this device
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "synchronising the stream: %s", cudaGetErrorString(e));
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, static_cast<uint32_t*>(base) + kCtrlError, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "reading the error word: %s", cudaGetErrorString(e));
+  if (word) {
+    e = cudaMemset(static_cast<uint32_t*>(base) + kCtrlError, 0, sizeof(word));
+    if (e != cudaSuccess) return set_error(ISA_ERR_CUDA, "clearing the error word: %s", cudaGetErrorString(e));
+    return set_error(ISA_ERR_TIMEOUT, "the allocation-free selection kernel's wait timed out (error word 0x%x)",
+                     word);
+  }
   return ISA_OK;
 }

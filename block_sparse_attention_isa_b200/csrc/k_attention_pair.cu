@@ -598,7 +598,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-bool attention_pair_supported(const Plan& p) { return p.dt == 0 && p.D == kD; }
+// The build checks that the kernel compiled to kLaunchRegs registers per thread, which its
+// warpgroup register split needs. A library built some other way that got another count runs its
+// calls on the single-CTA kernel instead (the launcher below refuses to launch it).
+bool attention_pair_regs_ok() {
+  static int cached[64] = {0};  // 0 unknown, 1 ok, 2 not ok
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!cached[dev]) {
+    cudaFuncAttributes fa;
+    cached[dev] = (cudaFuncGetAttributes(&fa, attention_pair_kernel) == cudaSuccess && fa.numRegs == kLaunchRegs)
+                      ? 1 : 2;
+  }
+  return cached[dev] == 1;
+}
+
+bool attention_pair_supported(const Plan& p) { return p.dt == 0 && p.D == kD && attention_pair_regs_ok(); }
 
 cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, void* out, const Plan& pl,
                                   const Work& w, cudaStream_t s, int* n_ctas) {

@@ -36,7 +36,9 @@
  *
  * Layout: q, k, v and out are row-major contiguous [B, H, N, D] with
  * N = L_src + L_ctx, in the element type given by isa_dtype (bfloat16 or
- * float32); out has the same type. Sizes supported: D in {64, 128}, b in
+ * float32); out has the same type. Device pointers must be 16-byte aligned
+ * (the kernels move them with bulk and tensor copies); a misaligned one is
+ * rejected with ISA_ERR_ARG before any GPU work. Sizes supported: D in {64, 128}, b in
  * {64, 128}, any positive L_src and L_ctx with n_src + n_ctx <= 2048;
  * float32 only with D = 64.
  *
@@ -67,7 +69,7 @@ typedef enum { ISA_BF16 = 0, ISA_F32 = 1 } isa_dtype;
 
 enum {
   ISA_OK = 0,
-  ISA_ERR_ARG = -1,         /* null or aliased pointer, non-positive size, ratio outside [0,1] or NaN */
+  ISA_ERR_ARG = -1,         /* null, aliased or misaligned pointer, non-positive size, ratio outside [0,1] or NaN */
   ISA_ERR_SHAPE = -2,       /* reserved: lengths that b does not divide are accepted (short last blocks) */
   ISA_ERR_UNSUPPORTED = -3, /* D, b, dtype or the block count outside the supported set */
   ISA_ERR_WORKSPACE = -4,   /* workspace null or smaller than isa_workspace_bytes() */
@@ -122,8 +124,12 @@ ISA_API int isa_forward(const void* q, const void* k, const void* v, int B, int 
 /*
  * isa_forward_host - the same pass with HOST buffers (pageable or pinned):
  * copies q, k, v to the device, runs the pass, copies out (and the optional
- * dbg_sel / dbg_route, host int32) back, then synchronises. Device memory is
- * allocated and freed inside the call. Element type as given by dt.
+ * dbg_sel / dbg_route, host int32) back, then synchronises. Element type as
+ * given by dt. Device memory is taken inside the call from a stream-ordered
+ * memory pool that belongs to the library (one per device, created on first
+ * use) and given back to that pool before returning; the pool keeps the memory
+ * for the next call until the process exits. The device's default pool and its
+ * settings are not touched.
  */
 ISA_API int isa_forward_host(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
                      float alpha_s, float alpha_f, isa_dtype dt, void* out, int32_t* dbg_sel, int32_t* dbg_route);
@@ -181,22 +187,37 @@ ISA_API int isa_set_stage_events(void* const* events, int n_events);
  * operator plugins that a host runtime hands only their input and output
  * buffers, or serving loops that forbid cudaMalloc because it can
  * synchronise the device.
- *   q, k, v    device inputs [B, H, N, D] (as for isa_forward_ex)
+ *   q, k, v    device inputs [B, H, N, D] (as for isa_forward_ex, 16-byte aligned)
  *   sel        device int32 [B, H, k] output: kept context blocks, ascending
- *   colscore   device float32 [B, H, N_ctx / b] output: context-block scores
+ *   colscore   device float32 [B, H, ceil(L_ctx / b)] output: context-block scores
  * Scratch (the block means of Q, K, V, 3 * B*H * n_q * D * 4 bytes, plus
  * small partial sums, counters and control words, each part rounded up to 256
  * bytes) lives in a fixed 32 MiB device array inside the library, which
  * every GPU that loads the library holds until the process exits. Larger sizes
  * return ISA_ERR_UNSUPPORTED before any GPU work. The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress); make that first
- * call before any stream capture. Every call shares the one array: calls whose
- * GPU work may overlap (several streams or host threads on one device) race on
- * it and must be serialised by the caller. No allocation is made.
+ * call before any stream capture. The looked-up address is kept for the life of
+ * the process and does not survive cudaDeviceReset: after a reset, this entry
+ * point must not be called again in that process. Every call shares the one
+ * array: calls whose GPU work may overlap (several streams or host threads on
+ * one device) race on it and must be serialised by the caller. No allocation is
+ * made. The return value covers the enqueue only; a kernel wait that gave up is
+ * reported by isa_select_context_noalloc_status, which the caller must check
+ * before the next call on the device (each call clears the array's error word).
  */
 ISA_API int isa_select_context_noalloc(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx,
                                        int D, int b, float alpha_s, isa_dtype dt, int32_t* sel, float* colscore,
                                        void* stream);
+
+/*
+ * isa_select_context_noalloc_status - companion of isa_select_context_noalloc
+ * (the paper has no counterpart). Synchronises `stream`, then reads and clears
+ * the error word in the library's fixed scratch array on the current device.
+ * Returns ISA_OK (also when no allocation-free call has run on the device),
+ * ISA_ERR_TIMEOUT when a bounded wait of the last call's kernel gave up (its
+ * sel and colscore are then not valid), or ISA_ERR_CUDA. Allocates nothing.
+ */
+ISA_API int isa_select_context_noalloc_status(void* stream);
 
 /* Number of kernel launches one isa_forward_ex call makes for these sizes (0 if invalid). */
 ISA_API int isa_launch_count(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, isa_dtype dt);
@@ -236,6 +257,15 @@ ISA_API int isa_forward_ns(const void* q, const void* k, const void* v, int B, i
                            int b, float alpha_s, float alpha_f, float alpha_ns, isa_dtype dt, void* out,
                            int32_t* dbg_sel, int32_t* dbg_route, int32_t* dbg_ns, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/*
+ * isa_forward_host_ns - isa_forward_host with the no-sparsity ratio alpha_ns
+ * (host buffers, copies inside the call, synchronous; alpha_ns as for
+ * isa_forward_ns). With alpha_ns = 0 it is isa_forward_host.
+ */
+ISA_API int isa_forward_host_ns(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx,
+                                int D, int b, float alpha_s, float alpha_f, float alpha_ns, isa_dtype dt, void* out,
+                                int32_t* dbg_sel, int32_t* dbg_route);
 
 /* Number of kernel launches one isa_forward_ns call makes for these sizes (0 if invalid). */
 ISA_API int isa_launch_count_ns(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f,

@@ -185,3 +185,34 @@ def test_ragged_block_counts(L, L_src, L_ctx, b):
     assert k == O.kept_context_blocks(0.5, n_ctx) and n_flat == O.taylor_block_count(0.5, n_q)
     # K_new takes b rows for every block, a short one padded
     assert isa.workspace_bytes(1, 1, L_src, L_ctx, 64, b, 0.5) > 0
+
+
+@pytest.mark.parametrize("which", ["q", "k", "v", "out"])
+def test_misaligned_device_pointers_are_argument_errors(L, which):
+    """Bulk and tensor copies need 16-byte aligned addresses: a misaligned pointer is rejected
+    before any CUDA call (no workspace is given, so a missed check would return -4 instead)."""
+    ptrs = dict(q=FAKE, k=FAKE + (1 << 32), v=FAKE + (2 << 32), out=FAKE + (3 << 32))
+    ptrs[which] += 2  # a bf16 element off the 16-byte grid
+    rc = _fwd(L, q=ptrs["q"], k=ptrs["k"], v=ptrs["v"], out=ptrs["out"])
+    assert rc == -1
+    assert "16-byte aligned" in isa.last_error() and which in isa.last_error()
+    rc = L.isa_forward_ns(ptrs["q"], ptrs["k"], ptrs["v"], 1, 2, 512, 512, 64, 64, 0.5, 0.5, 0.25, 0,
+                          ptrs["out"], None, None, None, None, 0, None)
+    assert rc == -1
+
+
+@pytest.mark.parametrize("which", ["q", "k", "v"])
+def test_noalloc_rejects_misaligned_inputs(L, which):
+    ptrs = dict(q=FAKE, k=FAKE + (1 << 32), v=FAKE + (2 << 32))
+    ptrs[which] += 8
+    rc = L.isa_select_context_noalloc(ptrs["q"], ptrs["k"], ptrs["v"], 1, 2, 512, 512, 64, 64, 0.5, 0,
+                                      FAKE + (3 << 32), FAKE + (4 << 32), None)
+    assert rc == -1
+    assert "16-byte aligned" in isa.last_error()
+
+
+def test_host_entry_points_take_unaligned_host_buffers(L):
+    """Host buffers are copied, so their alignment is free; argument errors still come first."""
+    rc = L.isa_forward_host_ns(FAKE + 2, FAKE + (1 << 32), FAKE + (2 << 32), 1, 2, 512, 512, 64, 64, 0.5, 1.5,
+                               0.25, 0, FAKE + (3 << 32), None, None)
+    assert rc == -1 and "alpha" in isa.last_error()

@@ -74,3 +74,28 @@ def test_flop_and_byte_counts_match_the_oracle():
     hb = bench.hbm_bytes_per_call(w)
     assert hb["pool"] == 3 * 40 * 32768 * 128 * 2
     assert hb["gather"] == 2 * 2 * 40 * 32 * 128 * 128 * 2
+
+
+def test_roofline_peak_follows_the_timed_region():
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"bf16_tflops": 1659.6, "bf16_tflops_sustained": 1382.4, "hbm_gbs": 6552.6}
+    # a 0.1 s timed region sits below the power cap's reaction time: the burst GEMM figure
+    assert bench.roofline_peak(peaks, 0.1) == (1659.6, "burst")
+    # a seconds-long one runs under the power cap: the sustained figure
+    assert bench.roofline_peak(peaks, 1.06) == (1382.4, "sustained")
+    assert bench.roofline_peak({"bf16_tflops": 1590.0}, 5.0) == (1590.0, "burst")
+
+
+def test_weak_scaling_units_differ_per_rank():
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    import isa_synth
+    w = isa_synth.Workload("u", 1, 2, 64, 256, 256, 64, 0.5, 0.5, 0.1, 1.0, 0.5, "f32")
+    q0 = bench.workload_inputs(w, batch=0)[0]
+    q1 = bench.workload_inputs(w, batch=1)[0]
+    assert q0.shape == q1.shape == (1, 2, 512, 64)
+    assert not np.array_equal(q0, q1)
+    # batch element r is the draw of slice (r, h) of the generator
+    np.testing.assert_array_equal(q1[0, 1], isa_synth.make_slice(w, 0, 1, 1, 0)[0])

@@ -6,8 +6,9 @@ their pooled rows with weight b, in one softmax (papernotes.org, Key designs 2
 and 3). Small workloads are compared in full against the float64 oracle: kept
 blocks, routing and the per-block exact-block lists bit-exactly (inputs whose
 choices lie within 1e-3 of a tie are redrawn), outputs within max-abs 2e-2 and
-relative L2 5e-3. The 32K-token workload is checked on sampled rows of the
-query blocks whose exact-block choice clears the same tie margin.
+relative L2 5e-3. The 32K-token workload is checked in every row of its first
+two heads (exact blocks, and the Taylor blocks whose exact-block choice clears
+the same tie margin) and on sampled rows of such blocks in the other heads.
 """
 import multiprocessing as mp
 import os
@@ -149,27 +150,38 @@ def test_alpha_ns_rejects_f32():
 ROWS_PER_BLOCK = 2
 BLOCKS_PER_HEAD = 6
 ALPHA_NS_FULL = 0.0625
+WHOLE_HEADS_NS = 2  # heads compared in every row of the exact blocks and the margin-clear Taylor blocks
 
 
 def _slice_work_ns(args):
-    """Worker: stages 1-3 of the oracle with alpha_ns, and sampled rows of margin-clear Taylor blocks."""
+    """Worker: stages 1-3 of the oracle with alpha_ns, then either the whole slice (rows of the
+    exact blocks and of every margin-clear Taylor block) or sampled rows of margin-clear Taylor blocks."""
     import sys
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     import isa_synth as S
     from oracle import isa_oracle as O
-    name, bi, h, attempt, a_ns, margin = args
+    from threadpoolctl import threadpool_limits
+    name, bi, h, attempt, a_ns, margin, whole, threads = args
     w = S.all_workloads()[name]
     q, k, v = S.make_slice(w, 0, bi, h, attempt)
-    sr = O.isa_select_route_ref(q, k, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, a_ns)
-    clear = np.array([i for i in sr["taylor"] if sr["ns_row_margin"][i] >= margin], np.int64)
-    rng = np.random.default_rng([bi, h, 11])
-    blk = rng.choice(clear, size=min(BLOCKS_PER_HEAD, len(clear)), replace=False) if len(clear) else clear
-    rows = np.array(sorted(int(i) * w.b + int(o) for i in blk for o in rng.integers(0, w.b, ROWS_PER_BLOCK)),
-                    np.int64)
-    rows = np.unique(rows)
-    ref_rows = O.isa_rows_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, rows, sr=sr, alpha_ns=a_ns)
+    with threadpool_limits(limits=threads):
+        sr = O.isa_select_route_ref(q, k, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, a_ns)
+        clear = np.array([i for i in sr["taylor"] if sr["ns_row_margin"][i] >= margin], np.int64)
+        if whole:
+            full = O.isa_slice_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, alpha_ns=a_ns)
+            blk = np.sort(np.concatenate([sr["exact"], clear]))
+            rows = (blk[:, None] * w.b + np.arange(w.b)[None, :]).ravel()
+            ref_rows = full["out"][rows]
+        else:
+            rng = np.random.default_rng([bi, h, 11])
+            blk = rng.choice(clear, size=min(BLOCKS_PER_HEAD, len(clear)), replace=False) if len(clear) else clear
+            rows = np.array(sorted(int(i) * w.b + int(o) for i in blk for o in rng.integers(0, w.b, ROWS_PER_BLOCK)),
+                            np.int64)
+            rows = np.unique(rows)
+            ref_rows = O.isa_rows_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, rows, sr=sr,
+                                      alpha_ns=a_ns)
     return (bi, h, q, k, v, sr["sel"], np.concatenate([sr["exact"], sr["taylor"]]), clear, sr["ns_sel"], rows,
-            ref_rows, len(sr["taylor"]))
+            ref_rows, len(sr["taylor"]), whole)
 
 
 def test_full_size_32k_alpha_ns():
@@ -180,10 +192,12 @@ def test_full_size_32k_alpha_ns():
     table = isa_synth.load_attempts()
     att = isa_synth.attempts_for(w, 0, table)
     assert att is not None
-    jobs = [(w.name, bi, h, int(att[bi, h]), ALPHA_NS_FULL, MARGIN) for bi in range(w.B) for h in range(w.H)]
+    threads_whole = max(1, (os.cpu_count() or 4) // WHOLE_HEADS_NS)
+    jobs = [(w.name, bi, h, int(att[bi, h]), ALPHA_NS_FULL, MARGIN, bi * w.H + h < WHOLE_HEADS_NS,
+             threads_whole if bi * w.H + h < WHOLE_HEADS_NS else 1) for bi in range(w.B) for h in range(w.H)]
     pool = mp.get_context("spawn").Pool(max(2, min(16, (os.cpu_count() or 4) - 1)))
     try:
-        res = pool.map(_slice_work_ns, jobs)
+        res = pool.map(_slice_work_ns, jobs, chunksize=1)
     finally:
         pool.terminate()
     dev = torch.device("cuda")
@@ -201,16 +215,22 @@ def test_full_size_32k_alpha_ns():
     o = out.float()
     assert bool(((o >= vmin - MAX_ABS) & (o <= vmax + MAX_ABS)).all())
     sel_h, route_h, ns_h, out_h = sel.cpu().numpy(), route.cpu().numpy(), ns.cpu().numpy(), o.cpu().numpy()
-    diffs, refs, n_clear, n_taylor = [], [], 0, 0
-    for bi, h, q, k, v, sel_ref, route_ref, clear, ns_ref, rows, ref_rows, nt in res:
+    diffs, refs, n_clear, n_taylor, n_whole = [], [], 0, 0, 0
+    for bi, h, q, k, v, sel_ref, route_ref, clear, ns_ref, rows, ref_rows, nt, whole in res:
         np.testing.assert_array_equal(sel_h[bi, h], sel_ref)
         np.testing.assert_array_equal(route_h[bi, h], route_ref)
         np.testing.assert_array_equal(ns_h[bi, h][clear], ns_ref[clear], err_msg=f"exact blocks, slice {bi},{h}")
         n_clear += len(clear)
         n_taylor += nt
-        if len(rows):
+        if whole:
+            n_whole += 1
+            d = out_h[bi, h, rows] - ref_rows
+            ma, rl = float(np.abs(d).max()), float(np.linalg.norm(d) / np.linalg.norm(ref_rows))
+            assert ma <= MAX_ABS and rl <= REL_L2, f"whole head {bi},{h}: max-abs {ma:.3e}, rel-L2 {rl:.3e}"
+        elif len(rows):
             diffs.append(out_h[bi, h, rows] - ref_rows)
             refs.append(ref_rows)
+    assert n_whole == WHOLE_HEADS_NS
     assert n_clear >= n_taylor // 2, (n_clear, n_taylor)
     d, r = np.concatenate(diffs), np.concatenate(refs)
     max_abs, rel = float(np.abs(d).max()), float(np.linalg.norm(d) / np.linalg.norm(r))

@@ -75,3 +75,58 @@ def test_ragged_full_parity(case):
                 np.testing.assert_array_equal(ns[r["taylor"]], r["ns_sel"][r["taylor"]])
             ref_out[bi, h] = r["out"]
     compare_out(out, ref_out)
+
+
+# ---------------------------------------------------------------- full size
+
+def _ragged_slice_work(args):
+    """Worker: the accepted draw of one slice and its whole-slice ragged oracle."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import isa_synth as S
+    from oracle import isa_oracle_ragged as RR
+    from threadpoolctl import threadpool_limits
+    w, bi, h, margin, threads = args
+    with threadpool_limits(limits=threads):
+        for a in range(64):
+            q, k, v = S.make_slice(w, 0, bi, h, a)
+            sr = RR.isa_select_route_ragged(q, k, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+            if min(sr["topk_margin"], sr["route_margin"]) >= margin:
+                break
+        else:
+            raise RuntimeError(f"no accepted attempt for slice {bi},{h}")
+        r = RR.isa_slice_ref_ragged(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, sr=sr)
+    return bi, h, q, k, v, r["sel"], r["route"], r["out"]
+
+
+def test_ragged_full_size_32k():
+    """The headline shape with both parts ragged: L_src = 16300 (127 blocks + 44 tokens),
+    L_ctx = 16500 (128 blocks + 116 tokens), b = 128, alpha_s = 0.25, alpha_f = 0.6, 4 heads,
+    every output row compared."""
+    import multiprocessing as mp
+    import os
+    import torch
+    import block_sparse_attention_isa_b200 as isa
+    w = isa_synth.Workload("ragged_n32800_b128", 1, 4, 128, 16300, 16500, 128, 0.25, 0.6, 0.1, 1.0, 0.5, "bf16")
+    threads = max(1, (os.cpu_count() or 4) // (w.B * w.H))
+    pool = mp.get_context("spawn").Pool(w.B * w.H)
+    try:
+        res = pool.map(_ragged_slice_work, [(w, bi, h, MARGIN, threads) for bi in range(w.B) for h in range(w.H)],
+                       chunksize=1)
+    finally:
+        pool.terminate()
+    shape = (w.B, w.H, w.N, w.D)
+    q, k, v = (np.zeros(shape, np.float32) for _ in range(3))
+    for bi, h, qs, ks, vs, *_ in res:
+        q[bi, h], k[bi, h], v[bi, h] = qs, ks, vs
+    tq, tk, tv = (to_device(x, w) for x in (q, k, v))
+    out, sel, route = isa.forward(tq, tk, tv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, debug=True)
+    isa.device_status()
+    out, sel, route = out.float().cpu().numpy(), sel.cpu().numpy(), route.cpu().numpy()
+    ref = np.zeros(shape, np.float64)
+    for bi, h, _, _, _, sel_ref, route_ref, out_ref in res:
+        np.testing.assert_array_equal(sel[bi, h], sel_ref, err_msg=f"kept blocks {bi},{h}")
+        np.testing.assert_array_equal(route[bi, h], route_ref, err_msg=f"routing {bi},{h}")
+        ref[bi, h] = out_ref
+    compare_out(out, ref)

@@ -494,3 +494,59 @@ def test_planted_mistake_in_mixed_path(monkeypatch):
     monkeypatch.setattr(O, "taylor_mixed_rows", _mixed_wrong)
     with pytest.raises(AssertionError):
         test_mixed_taylor_brute_force_loops()
+
+
+# ----------------------------------------------------------------------------- isa_rows_ref and no_sparse_margin
+# isa_rows_ref is the oracle behind every sampled full-size GPU comparison. It maps rows to
+# paths on its own (row // b in the Taylor set), so it is pinned to the whole-slice oracle,
+# which the pins above tie to closed forms, library routines and brute force.
+
+@pytest.mark.parametrize("b,a_s,a_f,a_ns", [(8, 0.5, 0.5, 0.0), (8, 0.25, 0.75, 0.0), (16, 1.0, 0.0, 0.0),
+                                            (8, 0.5, 1.0, 0.0), (8, 0.5, 0.5, 0.25), (16, 0.5, 0.625, 0.5)])
+def test_rows_ref_equals_slice_ref(b, a_s, a_f, a_ns):
+    w = _small(b=b, L_src=64, L_ctx=96, a_s=a_s, a_f=a_f)
+    q, k, v = isa_synth.make_slice(w, 11, 0, 0, 0)
+    full = O.isa_slice_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, alpha_ns=a_ns)
+    rng = np.random.default_rng(5)
+    # every row of two whole blocks, scattered rows, the first and the last row
+    rows = np.unique(np.concatenate([np.arange(b, 2 * b), np.arange(w.N - b, w.N),
+                                     rng.integers(0, w.N, 40), [0, w.N - 1]]))
+    got = O.isa_rows_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, rows, alpha_ns=a_ns)
+    np.testing.assert_allclose(got, full["out"][rows], rtol=0, atol=1e-13)
+    # the same with the stage 1-3 results passed in, as the GPU tests do
+    sr = O.isa_select_route_ref(q, k, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, a_ns)
+    got2 = O.isa_rows_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, rows, sr=sr, alpha_ns=a_ns)
+    np.testing.assert_array_equal(got2, got)
+    # all rows at once equal the whole slice
+    allr = O.isa_rows_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, np.arange(w.N), alpha_ns=a_ns)
+    np.testing.assert_allclose(allr, full["out"], rtol=0, atol=1e-13)
+
+
+def test_rows_ref_catches_a_row_to_block_slip(monkeypatch):
+    """A row mapped to the block of its neighbour takes the wrong path and fails the pin above."""
+    w = _small(b=8, L_src=64, L_ctx=96, a_s=0.5, a_f=0.5)
+    q, k, v = isa_synth.make_slice(w, 11, 0, 0, 0)
+    full = O.isa_slice_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+    sr = O.isa_select_route_ref(q, k, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+    taylor = set(int(t) for t in sr["taylor"])
+    # rows whose block and the next block take different paths
+    rows = np.array([i * w.b for i in range(w.N // w.b - 1) if (i in taylor) != (i + 1 in taylor)])
+    assert len(rows)
+    wrong = O.isa_rows_ref(q, k, v, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, rows + w.b, sr=sr)
+    assert np.abs(wrong - full["out"][rows]).max() > 1e-3
+
+
+def test_no_sparse_margin_closed_form():
+    p = np.array([[0.5, 0.3, 0.2],
+                  [0.1, 0.6, 0.3]])
+    # k_ns = 1: row 0 (0.5 - 0.3) / 0.5 = 0.4, row 1 (0.6 - 0.3) / 0.6 = 0.5 -> 0.4
+    assert O.no_sparse_margin(p, 1) == pytest.approx(0.4, abs=1e-15)
+    # k_ns = 2: row 0 (0.3 - 0.2) / 0.3 = 1/3, row 1 (0.3 - 0.1) / 0.3 = 2/3 -> 1/3
+    assert O.no_sparse_margin(p, 2) == pytest.approx(1.0 / 3.0, abs=1e-15)
+    # a tie at the boundary is a zero margin; no boundary (k_ns = 0 or all blocks) is infinite
+    assert O.no_sparse_margin(np.array([[0.4, 0.4, 0.2]]), 1) == 0.0
+    assert O.no_sparse_margin(p, 0) == math.inf
+    assert O.no_sparse_margin(p, 3) == math.inf
+    assert O.no_sparse_margin(np.zeros((0, 3)), 1) == math.inf
+    # the margin is invariant to the row order and to a common positive scale of a row
+    assert O.no_sparse_margin(p[::-1] * np.array([[3.0], [0.5]]), 1) == pytest.approx(0.4, abs=1e-15)
