@@ -55,13 +55,18 @@ def no_sparse_count(alpha_ns: float, n_new: int) -> int:
     return max(0, min(n_new, math.ceil(float(np.float32(alpha_ns)) * n_new - 1e-4)))
 
 
+def _cdiv(a: int, b: int) -> int:
+    return -(-a // b)
+
+
 def flops_per_call(w, alpha_ns: float = 0.0) -> dict:
     """Multiply-adds of each stage x 2 for one call over all B*H slices (the pass's own counts).
 
     With alpha_ns > 0 a Taylor query row attends to the n_new - k_ns pooled rows
-    and the k_ns * b keys of its exact blocks."""
-    N = w.L_src + w.L_ctx
-    n_q, n_src, n_ctx = N // w.b, w.L_src // w.b, w.L_ctx // w.b
+    and the k_ns * b keys of its exact blocks. With short last blocks (b dividing
+    neither length) every block counts b rows and b keys: the work the kernels execute."""
+    n_src, n_ctx = _cdiv(w.L_src, w.b), _cdiv(w.L_ctx, w.b)
+    n_q = n_src + n_ctx
     k = max(0, min(n_ctx, math.ceil(float(np.float32(w.alpha_s)) * n_ctx - 1e-4)))
     n_flat = max(0, min(n_q, math.floor(float(np.float32(w.alpha_f)) * n_q + 1e-4)))
     n_new = n_src + k
@@ -78,7 +83,7 @@ def hbm_bytes_per_call(w) -> dict:
     """Algorithmic HBM bytes of the pooling/top-k stage (read Q, K, V once) and the gather."""
     e = 2 if w.dtype == "bf16" else 4
     N = w.L_src + w.L_ctx
-    n_ctx = w.L_ctx // w.b
+    n_ctx = _cdiv(w.L_ctx, w.b)
     k = max(0, min(n_ctx, math.ceil(float(np.float32(w.alpha_s)) * n_ctx - 1e-4)))
     return dict(pool=3.0 * w.B * w.H * N * w.D * e, gather=2.0 * 2.0 * w.B * w.H * k * w.b * w.D * e)
 
@@ -206,14 +211,23 @@ def bf16_bits(x):
     return isa_synth.round_to_bf16_bits(x)
 
 
+def is_ragged(w) -> bool:
+    return bool(w.L_src % w.b or w.L_ctx % w.b)
+
+
 def cpu_oracle_sample(w, q, k, v, heads, seconds_cap=60.0, alpha_ns=0.0):
     """Run the oracle on some heads; returns (TFLOP/s, seconds, heads done)."""
     from oracle import isa_oracle as O
+    from oracle import isa_oracle_ragged as R
     f = flops_per_call(w, alpha_ns)["total"] / (w.B * w.H)
     t0 = time.perf_counter()
     done = 0
     for h in heads:
-        O.isa_slice_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, alpha_ns=alpha_ns)
+        if is_ragged(w):
+            R.isa_slice_ref_ragged(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, alpha_ns)
+        else:
+            O.isa_slice_ref(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f,
+                            alpha_ns=alpha_ns)
         done += 1
         if time.perf_counter() - t0 > seconds_cap:
             break
@@ -233,6 +247,8 @@ def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    if is_ragged(w):
+        return run_reference_whole_heads(args, w)
     import numpy as np
     from oracle import isa_oracle as O
     n_heads = min(w.B * w.H, max(1, args.steps + args.warmup))
@@ -278,6 +294,37 @@ def run_reference(args, w):
                        "N": w.N, "D": w.D, "b": w.b, "alpha_s": w.alpha_s, "alpha_f": w.alpha_f,
                        "alpha_ns": args.alpha_ns, "sample": sample},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_whole_heads(args, w):
+    """The reference arm for ragged lengths: each step is the ragged-length oracle over one
+    whole head of the workload (as it stands, on the host cores)."""
+    from oracle import isa_oracle_ragged as R
+    n_heads = min(w.B * w.H, max(1, args.steps + args.warmup))
+    q, k, v = isa_synth.make_inputs(w, 0, None, heads=[(0, h) for h in range(n_heads)])
+    per_head = flops_per_call(w, args.alpha_ns)["total"] / (w.B * w.H)
+
+    def step(s):
+        h = s % n_heads
+        R.isa_slice_ref_ragged(q[0, h], k[0, h], v[0, h], w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, args.alpha_ns)
+        return per_head
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    flops = sum(step(args.warmup + s) for s in range(args.steps))
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = f"per step: one whole head ({args.steps} steps over {n_heads} of {w.B * w.H} heads)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_label(args, w), "B": w.B, "H": w.H, "N": w.N, "D": w.D, "b": w.b,
+                       "alpha_s": w.alpha_s, "alpha_f": w.alpha_f, "alpha_ns": args.alpha_ns, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -473,7 +520,7 @@ def main():
     ap.add_argument("--heads", type=int, default=0,
                     help="run only the first H heads of the workload (small profiling captures; not a bench line)")
     args = ap.parse_args()
-    w = isa_synth.all_workloads()[args.workload]
+    w = {**isa_synth.all_workloads(), **isa_synth.RAGGED}[args.workload]
     args.full_workload = None
     if args.heads:
         args.full_workload = w

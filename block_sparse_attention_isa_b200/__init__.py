@@ -25,6 +25,8 @@ __all__ = [
     "forward",
     "forward_into",
     "forward_host",
+    "forward_varlen",
+    "varlen_workspace_bytes",
     "select_context_noalloc",
     "select_context_noalloc_status",
     "device_status",
@@ -65,6 +67,8 @@ EXPORTS = (
     "isa_select_context_noalloc",
     "isa_select_context_noalloc_status",
     "isa_forward_host_ns",
+    "isa_workspace_bytes_varlen",
+    "isa_forward_varlen",
     "isa_plan_ns",
     "isa_workspace_bytes_ns",
     "isa_forward_ns",
@@ -128,6 +132,11 @@ def lib() -> ctypes.CDLL:
     L.isa_select_context_noalloc_status.restype = c_int
     L.isa_forward_host_ns.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_float, c_float, c_int, vp, vp, vp]
     L.isa_forward_host_ns.restype = c_int
+    L.isa_workspace_bytes_varlen.argtypes = [c_int, c_int, vp, vp, c_int, c_int, c_float, c_int]
+    L.isa_workspace_bytes_varlen.restype = c_size
+    L.isa_forward_varlen.argtypes = [vp, vp, vp, c_int, c_int, vp, vp, c_int, c_int, c_float, c_float, c_int, vp, vp,
+                                     vp, vp, c_size, vp]
+    L.isa_forward_varlen.restype = c_int
     L.isa_plan_ns.argtypes = [c_int] * 6 + [c_float, c_float, c_float, i32p, i32p, i32p, i32p]
     L.isa_plan_ns.restype = c_int
     L.isa_workspace_bytes_ns.argtypes = [c_int] * 6 + [c_float, c_float, c_int]
@@ -323,6 +332,60 @@ def debug_pooled(B, H, L_src, L_ctx, D, b, alpha_s, dtype=ISA_BF16, workspace=No
                                   res["qc"].data_ptr(), res["kc"].data_ptr(), res["vc"].data_ptr(),
                                   res["colscore"].data_ptr(), res["sharp"].data_ptr(), s))
     return res
+
+
+def _i32_array(xs):
+    arr = (ctypes.c_int32 * len(xs))(*[int(x) for x in xs])
+    return arr
+
+
+def varlen_workspace_bytes(H, L_src, L_ctx, D, b, alpha_s, dtype=ISA_BF16) -> int:
+    """Workspace of isa_forward_varlen for the per-element length lists L_src, L_ctx."""
+    B = len(L_src)
+    if len(L_ctx) != B:
+        raise ValueError("L_src and L_ctx must have one entry per batch element")
+    n = lib().isa_workspace_bytes_varlen(B, H, _i32_array(L_src), _i32_array(L_ctx), D, b, alpha_s, dtype)
+    if n == 0:
+        raise IsaError(-1, last_error())
+    return n
+
+
+def forward_varlen(q, k, v, H: int, L_src, L_ctx, b: int, alpha_s: float, alpha_f: float, out=None,
+                   debug: bool = False, workspace=None, stream=None):
+    """The pass over a variable-length batch (isa_forward_varlen).
+
+    q, k, v: contiguous CUDA tensors holding the elements one after another, element i a
+    [H, L_src[i] + L_ctx[i], D] block (any outer shape; the last dimension is D). Returns out
+    (same shape), or (out, sel, route) with ``debug``: sel and route are 1-D int32 tensors holding
+    each element's [H, k_i] and [H, n_q_i] lists one after another.
+    """
+    torch = _torch()
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k and v must be contiguous CUDA tensors")
+    B, D = len(L_src), q.shape[-1]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    sel = route = None
+    if debug:
+        n_sel = n_route = 0
+        for ls, lc in zip(L_src, L_ctx):
+            n_q, kk, _ = plan(1, H, ls, lc, D, b, alpha_s, alpha_f)
+            n_sel += H * kk
+            n_route += H * n_q
+        sel = torch.empty(max(n_sel, 1), dtype=torch.int32, device=q.device)[:n_sel]
+        route = torch.empty(n_route, dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = _workspace(q.device, varlen_workspace_bytes(H, L_src, L_ctx, D, b, alpha_s, dt))
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    s = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    _check(lib().isa_forward_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, _i32_array(L_src),
+                                    _i32_array(L_ctx), D, b, alpha_s, alpha_f, dt, out.data_ptr(),
+                                    sel.data_ptr() if debug and sel.numel() else None,
+                                    route.data_ptr() if debug else None, workspace.data_ptr(), workspace.numel(), s))
+    return (out, sel, route) if debug else out
 
 
 def select_context_noalloc(q, k, v, L_src: int, L_ctx: int, b: int, alpha_s: float, sel, colscore, stream=None):

@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/isa.h"
 #include "isa_internal.h"
@@ -188,13 +189,14 @@ inline cudaError_t mark(int i, cudaStream_t s) {
   return g_stage_events_on ? cudaEventRecord(g_stage_events[i], s) : cudaSuccess;
 }
 
-// The CTA-pair attention kernel runs the calls it supports with whole blocks; calls with a
-// short last block take the single-CTA kernel, which masks the padding rows of K_new and
-// weighs short pooled rows by their length.
-bool use_pair_kernel(const Plan& p) { return attention_pair_supported(p) && !p.ragged; }
+// The CTA-pair attention kernel runs every call it supports (bf16, D = 128), whole blocks or
+// short last blocks alike; the single-CTA kernel runs D = 64 and float32.
+bool use_pair_kernel(const Plan& p) { return attention_pair_supported(p); }
 
+// keep_error: leave the error word as it is (a later element of a variable-length batch must not
+// clear what an earlier one reported)
 int run_forward(const void* q, const void* k, const void* v, const Plan& p, void* out, int32_t* dbg_sel,
-                int32_t* dbg_route, void* workspace, size_t workspace_bytes, cudaStream_t s) {
+                int32_t* dbg_route, void* workspace, size_t workspace_bytes, cudaStream_t s, bool keep_error = false) {
   const size_t need = workspace_layout(p, nullptr, nullptr);
   if (!workspace) return fail(ISA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
   if (workspace_bytes < need)
@@ -202,7 +204,9 @@ int run_forward(const void* q, const void* k, const void* v, const Plan& p, void
   if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(ISA_ERR_WORKSPACE, "workspace not 256-byte aligned");
   Work w;
   workspace_layout(p, &w, static_cast<char*>(workspace));
-  cudaError_t e = cudaMemsetAsync(w.ctrl, 0, sizeof(uint32_t) * (kCtrlWords + 2 * (size_t)p.BH), s);
+  static_assert(kCtrlError == 0, "the error word is the first control word");
+  const int skip = keep_error ? 1 : 0;
+  cudaError_t e = cudaMemsetAsync(w.ctrl + skip, 0, sizeof(uint32_t) * (kCtrlWords - skip + 2 * (size_t)p.BH), s);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace counters");
   if ((e = mark(0, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
   if ((e = launch_pool_score_topk(q, k, v, p, w, s)) != cudaSuccess) return cuda_fail(e, "pool/score/top-k launch");
@@ -353,6 +357,31 @@ int host_forward(const void* q, const void* k, const void* v, int B, int H, int 
   if (rc == ISA_OK && e != cudaSuccess) rc = cuda_fail(e, "releasing device buffers");
   return rc;
 }
+
+// Variable-length batches: element i of the batch is its own [1, H, N_i, D] call. Checks the
+// per-element arguments and returns the plans, the largest workspace and the element sizes.
+int varlen_plans(int B, int H, const int32_t* L_src, const int32_t* L_ctx, int D, int b, float alpha_s,
+                 float alpha_f, int dt, Plan* plans, size_t* ws_max, size_t* total_elems) {
+  if (B <= 0) return fail(ISA_ERR_ARG, "B must be positive (B=%d)", B);
+  if (!L_src || !L_ctx) return fail(ISA_ERR_ARG, "the length arrays L_src and L_ctx must not be NULL");
+  size_t mx = 0, tot = 0;
+  for (int i = 0; i < B; ++i) {
+    const int rc = make_plan(1, H, L_src[i], L_ctx[i], D, b, alpha_s, alpha_f, dt, &plans[i]);
+    if (rc != ISA_OK) {
+      char msg[512];
+      snprintf(msg, sizeof(msg), "%s", g_err);
+      return fail(rc, "batch element %d: %s", i, msg);
+    }
+    const size_t ws = workspace_layout(plans[i], nullptr, nullptr);
+    if (ws > mx) mx = ws;
+    tot += (size_t)H * plans[i].N * D;
+  }
+  if (ws_max) *ws_max = mx;
+  if (total_elems) *total_elems = tot;
+  return ISA_OK;
+}
+
+constexpr int kMaxVarlenBatch = 4096;
 
 }  // namespace
 }  // namespace isa
@@ -529,6 +558,63 @@ int isa_debug_pooled(int B, int H, int L_src, int L_ctx, int D, int b, float alp
     if (!c.dst) continue;
     cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToDevice, s);
     if (e != cudaSuccess) return cuda_fail(e, "copying pooled intermediates");
+  }
+  return ISA_OK;
+}
+
+}  // extern "C"
+
+extern "C" {
+
+size_t isa_workspace_bytes_varlen(int B, int H, const int32_t* L_src, const int32_t* L_ctx, int D, int b,
+                                  float alpha_s, isa_dtype dt) {
+  if (B > kMaxVarlenBatch) {
+    fail(ISA_ERR_UNSUPPORTED, "at most %d batch elements", kMaxVarlenBatch);
+    return 0;
+  }
+  std::vector<Plan> plans(B > 0 ? B : 1);
+  size_t ws = 0;
+  if (varlen_plans(B, H, L_src, L_ctx, D, b, alpha_s, 0.0f, (int)dt, plans.data(), &ws, nullptr) != ISA_OK) return 0;
+  return ws;
+}
+
+int isa_forward_varlen(const void* q, const void* k, const void* v, int B, int H, const int32_t* L_src,
+                       const int32_t* L_ctx, int D, int b, float alpha_s, float alpha_f, isa_dtype dt, void* out,
+                       int32_t* dbg_sel, int32_t* dbg_route, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (B > kMaxVarlenBatch) return fail(ISA_ERR_UNSUPPORTED, "at most %d batch elements", kMaxVarlenBatch);
+  std::vector<Plan> plans(B > 0 ? B : 1);
+  size_t ws_need = 0, total = 0;
+  int rc = varlen_plans(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, plans.data(), &ws_need, &total);
+  if (rc != ISA_OK) return rc;
+  // the whole packed batch: null, overlap and alignment checks over all elements at once
+  {
+    const size_t bytes = total * (size_t)plans[0].elem;
+    if (!q || !k || !v || !out) return fail(ISA_ERR_ARG, "q, k, v and out must not be NULL");
+    if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes))
+      return fail(ISA_ERR_ARG, "out must not overlap q, k or v");
+    if ((rc = check_aligned(q, k, v, out)) != ISA_OK) return rc;
+  }
+  if (!workspace) return fail(ISA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", ws_need);
+  if (workspace_bytes < ws_need)
+    return fail(ISA_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, ws_need);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  size_t off = 0, off_sel = 0, off_route = 0;
+  for (int i = 0; i < B; ++i) {
+    const Plan& p = plans[i];
+    const size_t e = off * p.elem;  // every element starts 16-byte aligned: H * N_i * D * elem, D a multiple of 16
+    rc = run_forward(static_cast<const char*>(q) + e, static_cast<const char*>(k) + e,
+                     static_cast<const char*>(v) + e, p, static_cast<char*>(out) + e,
+                     dbg_sel ? dbg_sel + off_sel : nullptr, dbg_route ? dbg_route + off_route : nullptr, workspace,
+                     workspace_bytes, s, /*keep_error=*/i > 0);
+    if (rc != ISA_OK) {
+      char msg[512];
+      snprintf(msg, sizeof(msg), "%s", g_err);
+      return fail(rc, "batch element %d: %s", i, msg);
+    }
+    off += (size_t)H * p.N * p.D;
+    off_sel += (size_t)H * p.k;
+    off_route += (size_t)H * p.n_q;
   }
   return ISA_OK;
 }

@@ -808,14 +808,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint64_t e;
             if (i % kPolyDen < kPolyNum) e = exp2_poly2(x);
             else e = pack2(ex2_approx(lo2(x)), ex2_approx(hi2(x)));
-            acc[i & 3] = fadd2(acc[i & 3], e);
             if constexpr (sizeof(T) == 2) {
               __nv_bfloat162 hv = __floats2bfloat162_rn(lo2(e), hi2(e));
               r[i] = *reinterpret_cast<uint32_t*>(&hv);
             } else {
+              acc[i & 3] = fadd2(acc[i & 3], e);
               r[2 * i] = static_cast<uint32_t>(e);
               r[2 * i + 1] = static_cast<uint32_t>(e >> 32);
             }
+          }
+          if constexpr (sizeof(T) == 2) {
+            // the row sum adds the same bf16 values that the P V MMA multiplies: with the lazy
+            // maximum the dominant keys' p lie in (1, 2^8] and round in bf16, and a sum of the
+            // unrounded p would leave numerator and denominator up to 2^-9 apart on them
+#pragma unroll
+            for (int i = half * kCols / 4; i < (half + 1) * kCols / 4; ++i)
+              acc[i & 1] = fadd2(acc[i & 1], pack2(__uint_as_float(r[i] << 16), __uint_as_float(r[i] & 0xffff0000u)));
           }
           // this half's P: bf16 pairs in kCols/4 columns, or fp32 in kCols/2 columns
           constexpr int kPCols = sizeof(T) == 2 ? kCols / 4 : kCols / 2;

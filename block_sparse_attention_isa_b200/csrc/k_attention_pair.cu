@@ -43,6 +43,12 @@
 //  * every wait is bounded; on a timeout the CTA flags an error in the device
 //    error word and in the abort flags of both CTAs, lets its copies land,
 //    meets its peer at a cluster barrier and frees TMEM.
+// Short last blocks (b does not divide L_src or L_ctx): K_new still gives every
+// block b rows, so the source part of K_new ends at n_src * b; the exact path
+// masks the rows past a short block's keys (the source part's padding and the
+// tail of a kept short context block), the Taylor path adds log2(len / b) to the
+// exponent of a short block's pooled row so that it weighs its own length, and
+// query rows are read and written by block start, only a block's own rows stored.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 #include <float.h>
@@ -90,6 +96,10 @@ struct PairParams {
   const int32_t* route;
   void* out;
   uint32_t* err;
+  // short blocks: sel [BH, k] kept context blocks (a kept short block is the last one kept)
+  const int32_t* sel;
+  int k, n_src, L_srcp, len_src_last, len_ctx_last, ragged;
+  float src_last_bias, ctx_last_bias;  // log2(len / b) / scale_log2: raw-score offsets of short pooled rows
   int BH, N, b, L_src, n_q, n_exact, n_flat, L_new, n_new;
   int bpt;      // blocks per 128-row tile (128 / b)
   int bpi;      // blocks per work item (4 tiles)
@@ -189,6 +199,33 @@ __device__ __forceinline__ int schedule(const PairParams& p, int pair, int npair
   if (pair < busy) return -1;
   const int g = (pair - busy) + (k - n_exact) * (npairs - busy);
   return g < T ? E + g : -1;
+}
+
+// First token of query block i (source blocks from 0, context blocks from L_src) and its length.
+__device__ __forceinline__ int qblock_start(const PairParams& p, int i) {
+  return i < p.n_src ? i * p.b : p.L_src + (i - p.n_src) * p.b;
+}
+__device__ __forceinline__ int qblock_len(const PairParams& p, int i) {
+  return i == p.n_src - 1 ? p.len_src_last : (i == p.n_q - 1 ? p.len_ctx_last : p.b);
+}
+// Whether head bh keeps the short last context block, which is then the last block of K_new.
+__device__ __forceinline__ bool short_ctx_kept(const PairParams& p, int bh) {
+  return p.len_ctx_last < p.b && p.k > 0 && __ldg(p.sel + (size_t)bh * p.k + p.k - 1) == p.n_q - p.n_src - 1;
+}
+// -inf for the key rows [lo, hi) of the 64-key tile starting at row `base` (uniform per tile).
+__device__ __forceinline__ void mask_key_rows(uint32_t (&r)[kCols], int base, int lo, int hi) {
+  if (hi <= base || lo >= base + kBN) return;
+#pragma unroll
+  for (int i = 0; i < kCols; ++i)
+    if (base + i >= lo && base + i < hi) r[i] = 0xff800000u;
+}
+// Adds `delta` to the raw score of the column holding pooled row `col` (tile rows from `base`).
+__device__ __forceinline__ void add_col_bias(uint32_t (&r)[kCols], int base, int col, float delta) {
+  const int c = col - base;
+  if (c < 0 || c >= kBN) return;
+#pragma unroll
+  for (int i = 0; i < kCols; ++i)
+    if (i == c) r[i] = __float_as_uint(__uint_as_float(r[i]) + delta);
 }
 
 struct Item {
@@ -334,7 +371,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int r = 64 * h;
             int u = ut * p.bpt + r / p.b;
             if (u >= it.nblk) u = ut * p.bpt;  // missing block of a partial tile: rows are not stored
-            const int y = it.blk(u) * p.b + (r % p.b);
+            const int y = qblock_start(p, it.blk(u)) + (r % p.b);  // rows past a short block: not stored
 #pragma unroll
             for (int c = 0; c < 2; ++c)
               tma_load_pair(sQ + t * kQTile + c * kQCh + h * 8192, &tm_q, q_full_l + 8u * t, c * 64, y, it.bh);
@@ -351,13 +388,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           if (rank == 0) mbar_arrive_expect_tx(&bars->kv_full[st], 2 * (kKHalf + kVHalf));
           const uint32_t bar = kv_full_l + 8u * st;
-          // K: this CTA's 32 keys of the tile (a 64-key tile never straddles the source/context seam)
+          // K: this CTA's 32 keys of the tile (a 64-key tile never straddles the seam of K_new's
+          // source part, which ends at n_src * b)
           {
             const int rk = r0 + (int)rank * kKRows;
             const CUtensorMap* map;
             int y;
             if (it.kind == 0) {
-              if (rk < p.L_src) { map = &tm_k; y = rk; } else { map = &tm_ksel; y = rk - p.L_src; }
+              if (rk < p.L_srcp) { map = &tm_k; y = rk; } else { map = &tm_ksel; y = rk - p.L_srcp; }
             } else {
               map = &tm_kcn; y = rk;
             }
@@ -369,7 +407,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const CUtensorMap* map;
             int y;
             if (it.kind == 0) {
-              if (r0 < p.L_src) { map = &tm_v; y = r0; } else { map = &tm_vsel; y = r0 - p.L_src; }
+              if (r0 < p.L_srcp) { map = &tm_v; y = r0; } else { map = &tm_vsel; y = r0 - p.L_srcp; }
             } else {
               map = &tm_vcn; y = r0;
             }
@@ -502,6 +540,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int k = 0, g = schedule(p, pair, npairs, 0); g >= 0 && ok; g = schedule(p, pair, npairs, ++k)) {
       const Item it = decode_item(p, g);
       if (t >= it.nslots) continue;
+      const bool cs = p.ragged ? short_ctx_kept(p, it.bh) : false;
       float m = -FLT_MAX, l = 0.f;
       for (int j = 0; j < it.nkv; ++j, ++seq) {
         const uint32_t buf = t_s + (seq & 1) * kBN;
@@ -514,6 +553,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kCols; ++i)
             if (i >= it.last_valid) r[i] = __float_as_uint(-INFINITY);
+        }
+        if (p.ragged) {  // (uniform branch; the first tile always holds a key of block 0)
+          if (it.kind == 0) {
+            // exact path: the padding rows of the short source block and of a kept short
+            // context block (the last block of K_new)
+            mask_key_rows(r, j * kBN, p.L_src, p.L_srcp);
+            if (cs) mask_key_rows(r, j * kBN, p.L_new - (p.b - p.len_ctx_last), p.L_new);
+          } else {
+            // Taylor path: a short block's pooled row weighs its own length
+            if (p.len_src_last < p.b) add_col_bias(r, j * kBN, p.n_src - 1, p.src_last_bias);
+            if (cs) add_col_bias(r, j * kBN, p.n_new - 1, p.ctx_last_bias);
+          }
         }
         // row max: 8 independent chains of 3-input max over the 64 scores
         float mc[8];
@@ -543,7 +594,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tmem_st32(t_o + 32 * c, o);
           }
         }
-        // p = 2^(s * scale - m) in pairs, written over this tile's S buffer as bf16 pairs
+        // p = 2^(s * scale - m) in pairs, written over this tile's S buffer as bf16 pairs. The row
+        // sum adds the same bf16 values that the P V MMA multiplies: with the lazy maximum, the
+        // dominant keys' p lie in (1, 2^8] and round in bf16, and a sum of the unrounded p would
+        // leave numerator and denominator up to 2^-9 apart on them
         const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(-m, -m);
         uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -551,9 +605,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint64_t x =
               ffma2(static_cast<uint64_t>(r[2 * i]) | (static_cast<uint64_t>(r[2 * i + 1]) << 32), sc2, nm2);
           const uint64_t e = (i % kPolyDen < kPolyNum) ? exp2_poly2(x) : pack2(ex2_approx(lo2(x)), ex2_approx(hi2(x)));
-          acc[i & 3] = fadd2(acc[i & 3], e);
           __nv_bfloat162 hv = __floats2bfloat162_rn(lo2(e), hi2(e));
-          r[i] = *reinterpret_cast<uint32_t*>(&hv);
+          const uint32_t hb = *reinterpret_cast<uint32_t*>(&hv);
+          r[i] = hb;
+          acc[i & 3] = fadd2(acc[i & 3], pack2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u)));
         }
         tmem_st32(buf, r);
         tmem_st_wait();
@@ -568,8 +623,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!pv_done(seq - 1)) { ok = false; break; }
       const int ut = 2 * t + (int)rank;
       const int u = ut * p.bpt + row / p.b;
-      const bool store = (ut < it.ntiles) && (u < it.nblk);
-      const size_t token = (size_t)it.blk(store ? u : 0) * p.b + (row % p.b);
+      const int qb = it.blk((ut < it.ntiles && u < it.nblk) ? u : 0);
+      const bool store = (ut < it.ntiles) && (u < it.nblk) && (row % p.b) < qblock_len(p, qb);
+      const size_t token = (size_t)qblock_start(p, qb) + (row % p.b);
       __nv_bfloat16* dst = out + ((size_t)it.bh * p.N + token) * kD;
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
@@ -630,12 +686,21 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
   p.n_flat = pl.n_flat;
   p.L_new = pl.L_new;
   p.n_new = pl.n_new;
+  p.sel = w.sel;
+  p.k = pl.k;
+  p.n_src = pl.n_src;
+  p.L_srcp = pl.L_srcp;
+  p.len_src_last = pl.len_src_last;
+  p.len_ctx_last = pl.len_ctx_last;
+  p.ragged = pl.ragged;
   p.bpt = kBM / pl.b;
   p.bpi = 4 * p.bpt;
   p.items_e = (pl.n_exact + p.bpi - 1) / p.bpi;
   p.items_t = (pl.n_flat + p.bpi - 1) / p.bpi;
   p.total = pl.BH * (p.items_e + p.items_t);
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+  p.src_last_bias = log2f((float)pl.len_src_last / (float)pl.b) / p.scale_log2;
+  p.ctx_last_bias = log2f((float)pl.len_ctx_last / (float)pl.b) / p.scale_log2;
   if (n_ctas) *n_ctas = 0;
   if (p.total == 0) return cudaSuccess;
 

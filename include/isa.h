@@ -271,6 +271,41 @@ ISA_API int isa_forward_host_ns(const void* q, const void* k, const void* v, int
 ISA_API int isa_launch_count_ns(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f,
                                 float alpha_ns, isa_dtype dt);
 
+/*
+ * Variable-length batches (papernotes.org, Key design 1 counts the context
+ * blocks as ceil(L_ctx / b), so every element of a batch may have its own
+ * lengths and its own short last blocks). Element i has L_src[i] source and
+ * L_ctx[i] context tokens, N_i = L_src[i] + L_ctx[i]; every element is an
+ * independent ISA pass over its H heads (its own pooling probe, top-k, routing
+ * and attention).
+ *
+ * isa_workspace_bytes_varlen - workspace for isa_forward_varlen: the largest
+ * element's isa_workspace_bytes (0 if an argument is invalid).
+ */
+ISA_API size_t isa_workspace_bytes_varlen(int B, int H, const int32_t* L_src, const int32_t* L_ctx, int D, int b,
+                                          float alpha_s, isa_dtype dt);
+
+/*
+ * isa_forward_varlen - the pass over a batch of B elements of different lengths.
+ *   L_src, L_ctx  HOST int32 arrays [B] (read during the call only); B <= 4096
+ *   q, k, v, out  device, packed: element i is a contiguous row-major [H, N_i, D]
+ *                 array starting at element offset H * D * (N_0 + ... + N_{i-1})
+ *                 (16-byte aligned, out not overlapping the inputs)
+ *   dbg_sel       optional device int32: element i's [H, k_i] kept context blocks,
+ *                 packed after those of the earlier elements; NULL to skip
+ *   dbg_route     optional device int32: element i's [H, n_q_i] routing, packed
+ *                 likewise; NULL to skip
+ *   workspace     at least isa_workspace_bytes_varlen() bytes: the elements run
+ *                 one after another on `stream` and reuse it
+ * Other arguments as for isa_forward_ex; errors name the failing element.
+ * Asynchronous; an element's kernel timeout stays in the workspace's error word
+ * for isa_device_status (later elements do not clear it).
+ */
+ISA_API int isa_forward_varlen(const void* q, const void* k, const void* v, int B, int H, const int32_t* L_src,
+                               const int32_t* L_ctx, int D, int b, float alpha_s, float alpha_f, isa_dtype dt,
+                               void* out, int32_t* dbg_sel, int32_t* dbg_route, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
 /* Message of the last failed call on this host thread ("" if none). */
 ISA_API const char* isa_last_error(void);
 

@@ -37,6 +37,7 @@ import numpy as np
 __all__ = [
     "Workload",
     "WORKLOADS",
+    "RAGGED",
     "SWEEP_51K",
     "sweep_workloads",
     "make_slice",
@@ -84,6 +85,13 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 HEADLINE = "bf16_n32768_b128"
+
+# The headline shape with lengths that b = 128 divides in neither part (a short last block in the
+# source part, 44 tokens, and in the context part, 116 tokens): a benchmark of ragged lengths.
+RAGGED: Dict[str, Workload] = {
+    "bf16_n32800_b128_ragged": Workload("bf16_n32800_b128_ragged", 1, 40, 128, 16300, 16500, 128, 0.25, 0.6, 0.1,
+                                        1.0, 0.5, "bf16"),
+}
 
 _SWEEP_BASE = Workload("bf16_n51200_b128", 1, 40, 128, 25600, 25600, 128, 0.25, 0.5, 0.1, 1.0, 0.5, "bf16")
 SWEEP_51K_ALPHA_S = (0.1, 0.25, 0.5)

@@ -216,3 +216,48 @@ def test_host_entry_points_take_unaligned_host_buffers(L):
     rc = L.isa_forward_host_ns(FAKE + 2, FAKE + (1 << 32), FAKE + (2 << 32), 1, 2, 512, 512, 64, 64, 0.5, 1.5,
                                0.25, 0, FAKE + (3 << 32), None, None)
     assert rc == -1 and "alpha" in isa.last_error()
+
+
+def _arr(xs):
+    import ctypes
+    return (ctypes.c_int32 * len(xs))(*xs)
+
+
+def test_varlen_workspace_is_the_largest_element(L):
+    Ls, Lc = [1000, 4096, 513], [1100, 4096, 700]
+    per = [isa.workspace_bytes(1, 2, a, c, 128, 128, 0.25) for a, c in zip(Ls, Lc)]
+    assert isa.varlen_workspace_bytes(2, Ls, Lc, 128, 128, 0.25) == max(per)
+
+
+@pytest.mark.parametrize("Ls,Lc,code,msg", [
+    ([512, 0], [512, 512], -1, "batch element 1"),       # an empty source part
+    ([512, 512], [512, -3], -1, "batch element 1"),
+    ([512], [512 * 4096], -3, "batch element 0"),         # block count above 2048
+])
+def test_varlen_rejects_bad_elements(L, Ls, Lc, code, msg):
+    rc = L.isa_forward_varlen(FAKE, FAKE + (1 << 32), FAKE + (2 << 32), len(Ls), 2, _arr(Ls), _arr(Lc), 64, 64,
+                              0.5, 0.5, 0, FAKE + (3 << 32), None, None, None, 0, None)
+    assert rc == code
+    assert msg in isa.last_error()
+
+
+def test_varlen_argument_errors(L):
+    # no length arrays
+    assert L.isa_forward_varlen(FAKE, FAKE, FAKE, 2, 2, None, None, 64, 64, 0.5, 0.5, 0, FAKE, None, None, None, 0,
+                                None) == -1
+    # B = 0
+    assert L.isa_forward_varlen(FAKE, FAKE, FAKE, 0, 2, _arr([1]), _arr([1]), 64, 64, 0.5, 0.5, 0, FAKE, None, None,
+                                None, 0, None) == -1
+    # out overlapping q over the packed batch (the second element reaches into out)
+    Ls, Lc = [512, 512], [512, 512]
+    assert L.isa_forward_varlen(FAKE, FAKE + (1 << 32), FAKE + (2 << 32), 2, 2, _arr(Ls), _arr(Lc), 64, 64, 0.5,
+                                0.5, 0, FAKE + 2 * 1024 * 64 * 2, None, None, None, 0, None) == -1
+    # misaligned v, then a missing workspace
+    assert L.isa_forward_varlen(FAKE, FAKE + (1 << 32), FAKE + (2 << 32) + 4, 2, 2, _arr(Ls), _arr(Lc), 64, 64, 0.5,
+                                0.5, 0, FAKE + (3 << 32), None, None, None, 0, None) == -1
+    assert L.isa_forward_varlen(FAKE, FAKE + (1 << 32), FAKE + (2 << 32), 2, 2, _arr(Ls), _arr(Lc), 64, 64, 0.5,
+                                0.5, 0, FAKE + (3 << 32), None, None, None, 0, None) == -4
+    # more elements than supported
+    big = [64] * 5000
+    assert L.isa_forward_varlen(FAKE, FAKE, FAKE, 5000, 1, _arr(big), _arr(big), 64, 64, 0.5, 0.5, 0, FAKE, None,
+                                None, None, 0, None) == -3

@@ -99,3 +99,22 @@ def test_weak_scaling_units_differ_per_rank():
     assert not np.array_equal(q0, q1)
     # batch element r is the draw of slice (r, h) of the generator
     np.testing.assert_array_equal(q1[0, 1], isa_synth.make_slice(w, 0, 1, 1, 0)[0])
+
+
+def test_ragged_workload_counts_by_hand():
+    sys.path.insert(0, ROOT)
+    import bench
+    import isa_synth
+    from oracle import isa_oracle_ragged as R
+    w = isa_synth.RAGGED["bf16_n32800_b128_ragged"]
+    assert bench.is_ragged(w) and not bench.is_ragged(isa_synth.WORKLOADS["bf16_n32768_b128"])
+    # ceil(16300 / 128) = 128 source and ceil(16500 / 128) = 129 context blocks; k = ceil(0.25 * 129) = 33,
+    # n_flat = floor(0.6 * 257) = 154, n_new = 161; every block counts b rows and b keys
+    n_q, k, n_flat, n_new = 257, 33, 154, 161
+    assert len(R.block_bounds(w.L_src, w.L_ctx, w.b)) == n_q
+    f = bench.flops_per_call(w)
+    assert f["exact"] == 4.0 * (n_q - n_flat) * 128 * n_new * 128 * 128 * 40
+    assert f["taylor"] == 4.0 * n_flat * 128 * n_new * 128 * 40
+    assert f["coarse"] == 2.0 * 128 * n_q * 128 * 40 and f["route"] == 2.0 * n_q * n_new * 128 * 40
+    hb = bench.hbm_bytes_per_call(w)
+    assert hb["pool"] == 3 * 40 * 32800 * 128 * 2 and hb["gather"] == 2 * 2 * 40 * k * 128 * 128 * 2
