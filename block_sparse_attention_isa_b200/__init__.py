@@ -27,6 +27,8 @@ __all__ = [
     "forward_host",
     "forward_varlen",
     "varlen_workspace_bytes",
+    "forward_train",
+    "backward",
     "select_context_noalloc",
     "select_context_noalloc_status",
     "device_status",
@@ -69,6 +71,9 @@ EXPORTS = (
     "isa_forward_host_ns",
     "isa_workspace_bytes_varlen",
     "isa_forward_varlen",
+    "isa_forward_train",
+    "isa_backward_workspace_bytes",
+    "isa_backward",
     "isa_plan_ns",
     "isa_workspace_bytes_ns",
     "isa_forward_ns",
@@ -137,6 +142,13 @@ def lib() -> ctypes.CDLL:
     L.isa_forward_varlen.argtypes = [vp, vp, vp, c_int, c_int, vp, vp, c_int, c_int, c_float, c_float, c_int, vp, vp,
                                      vp, vp, c_size, vp]
     L.isa_forward_varlen.restype = c_int
+    L.isa_forward_train.argtypes = [vp, vp, vp] + [c_int] * 6 + [c_float, c_float, c_int, vp, vp, vp, c_size, vp]
+    L.isa_forward_train.restype = c_int
+    L.isa_backward_workspace_bytes.argtypes = [c_int] * 6 + [c_float, c_int]
+    L.isa_backward_workspace_bytes.restype = c_size
+    L.isa_backward.argtypes = [vp] * 6 + [c_int] * 6 + [c_float, c_float, c_int, vp, vp, vp, vp, c_size, vp, c_size,
+                                                          vp]
+    L.isa_backward.restype = c_int
     L.isa_plan_ns.argtypes = [c_int] * 6 + [c_float, c_float, c_float, i32p, i32p, i32p, i32p]
     L.isa_plan_ns.restype = c_int
     L.isa_workspace_bytes_ns.argtypes = [c_int] * 6 + [c_float, c_float, c_int]
@@ -355,7 +367,7 @@ def forward_varlen(q, k, v, H: int, L_src, L_ctx, b: int, alpha_s: float, alpha_
     """The pass over a variable-length batch (isa_forward_varlen).
 
     q, k, v: contiguous CUDA tensors holding the elements one after another, element i a
-    [H, L_src[i] + L_ctx[i], D] block (any outer shape; the last dimension is D). Returns out
+    [H, L_src[i] + L_ctx[i], D] block (at least 2-D; the last dimension is D). Returns out
     (same shape), or (out, sel, route) with ``debug``: sel and route are 1-D int32 tensors holding
     each element's [H, k_i] and [H, n_q_i] lists one after another.
     """
@@ -363,6 +375,8 @@ def forward_varlen(q, k, v, H: int, L_src, L_ctx, b: int, alpha_s: float, alpha_
     for t in (q, k, v):
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError("q, k and v must be contiguous CUDA tensors")
+    if q.dim() < 2:
+        raise ValueError("q, k and v must be at least 2-D with D as the last dimension")
     B, D = len(L_src), q.shape[-1]
     dt = _dtype_code(q)
     if out is None:
@@ -386,6 +400,47 @@ def forward_varlen(q, k, v, H: int, L_src, L_ctx, b: int, alpha_s: float, alpha_
                                     sel.data_ptr() if debug and sel.numel() else None,
                                     route.data_ptr() if debug else None, workspace.data_ptr(), workspace.numel(), s))
     return (out, sel, route) if debug else out
+
+
+def forward_train(q, k, v, L_src: int, L_ctx: int, b: int, alpha_s: float, alpha_f: float, stream=None):
+    """Training forward (isa_forward_train): returns (out, lse, workspace).
+
+    lse float32 [B, H, N] is each row's log softmax denominator; the workspace (a fresh tensor,
+    not the module's shared one) holds the call's decisions and must be passed to ``backward``."""
+    torch = _torch()
+    B, H, N, D = q.shape
+    dt = _dtype_code(q)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    ws = torch.empty(workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dt), dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    s = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    _check(lib().isa_forward_train(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, L_src, L_ctx, D, b, alpha_s,
+                                   alpha_f, dt, out.data_ptr(), lse.data_ptr(), ws.data_ptr(), ws.numel(), s))
+    return out, lse, ws
+
+
+def backward(q, k, v, out, lse, dout, workspace, L_src: int, L_ctx: int, b: int, alpha_s: float, alpha_f: float,
+             stream=None, bwd_workspace=None):
+    """Gradients (dq, dk, dv) of sum(out * dout), from a forward_train call's tensors and workspace."""
+    torch = _torch()
+    B, H, N, D = q.shape
+    dt = _dtype_code(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nb = lib().isa_backward_workspace_bytes(B, H, L_src, L_ctx, D, b, alpha_s, dt)
+    if nb == 0:
+        raise IsaError(-1, last_error())
+    if bwd_workspace is None or bwd_workspace.numel() < nb:
+        bwd_workspace = torch.empty(nb, dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    s = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    _check(lib().isa_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                              dout.data_ptr(), B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, dt, dq.data_ptr(),
+                              dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                              bwd_workspace.data_ptr(), bwd_workspace.numel(), s))
+    return dq, dk, dv
 
 
 def select_context_noalloc(q, k, v, L_src: int, L_ctx: int, b: int, alpha_s: float, sel, colscore, stream=None):

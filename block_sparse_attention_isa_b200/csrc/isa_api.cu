@@ -111,6 +111,12 @@ bool overlaps(const void* a, const void* b, size_t bytes) {
   const char* y = static_cast<const char*>(b);
   return x < y + bytes && y < x + bytes;
 }
+// [a, a + na) and [b, b + nb) share a byte
+bool overlaps2(const void* a, size_t na, const void* b, size_t nb) {
+  const char* x = static_cast<const char*>(a);
+  const char* y = static_cast<const char*>(b);
+  return x < y + nb && y < x + na;
+}
 
 }  // namespace
 
@@ -196,7 +202,8 @@ bool use_pair_kernel(const Plan& p) { return attention_pair_supported(p); }
 // keep_error: leave the error word as it is (a later element of a variable-length batch must not
 // clear what an earlier one reported)
 int run_forward(const void* q, const void* k, const void* v, const Plan& p, void* out, int32_t* dbg_sel,
-                int32_t* dbg_route, void* workspace, size_t workspace_bytes, cudaStream_t s, bool keep_error = false) {
+                int32_t* dbg_route, void* workspace, size_t workspace_bytes, cudaStream_t s, bool keep_error = false,
+                float* lse = nullptr) {
   const size_t need = workspace_layout(p, nullptr, nullptr);
   if (!workspace) return fail(ISA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
   if (workspace_bytes < need)
@@ -204,6 +211,7 @@ int run_forward(const void* q, const void* k, const void* v, const Plan& p, void
   if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(ISA_ERR_WORKSPACE, "workspace not 256-byte aligned");
   Work w;
   workspace_layout(p, &w, static_cast<char*>(workspace));
+  w.lse = lse;
   static_assert(kCtrlError == 0, "the error word is the first control word");
   const int skip = keep_error ? 1 : 0;
   cudaError_t e = cudaMemsetAsync(w.ctrl + skip, 0, sizeof(uint32_t) * (kCtrlWords - skip + 2 * (size_t)p.BH), s);
@@ -617,6 +625,73 @@ int isa_forward_varlen(const void* q, const void* k, const void* v, int B, int H
     off_route += (size_t)H * p.n_q;
   }
   return ISA_OK;
+}
+
+}  // extern "C"
+
+extern "C" {
+
+int isa_forward_train(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
+                      float alpha_s, float alpha_f, isa_dtype dt, void* out, float* lse, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  Plan p;
+  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p);
+  if (rc != ISA_OK) return rc;
+  if ((rc = check_device_io(q, k, v, out, p)) != ISA_OK) return rc;
+  if (!lse) return fail(ISA_ERR_ARG, "lse must not be NULL");
+  if (reinterpret_cast<uintptr_t>(lse) & 15) return fail(ISA_ERR_ARG, "lse must be 16-byte aligned");
+  const size_t lse_bytes = sizeof(float) * (size_t)p.BH * p.N, io = (size_t)p.BH * p.N * p.D * p.elem;
+  if (overlaps2(lse, lse_bytes, q, io) || overlaps2(lse, lse_bytes, k, io) || overlaps2(lse, lse_bytes, v, io) ||
+      overlaps2(lse, lse_bytes, out, io) || overlaps2(lse, lse_bytes, workspace, workspace_bytes))
+    return fail(ISA_ERR_ARG, "lse must not overlap q, k, v, out or the workspace");
+  return run_forward(q, k, v, p, out, nullptr, nullptr, workspace, workspace_bytes, static_cast<cudaStream_t>(stream),
+                     false, lse);
+}
+
+size_t isa_backward_workspace_bytes(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, isa_dtype dt) {
+  Plan p;
+  if (make_plan(B, H, L_src, L_ctx, D, b, alpha_s, 0.0f, (int)dt, &p) != ISA_OK) return 0;
+  return backward_workspace_bytes(p);
+}
+
+int isa_backward(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+                 int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s, float alpha_f, isa_dtype dt,
+                 void* dq, void* dk, void* dv, void* fwd_workspace, size_t fwd_workspace_bytes, void* bwd_workspace,
+                 size_t bwd_workspace_bytes, void* stream) {
+  Plan p;
+  int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p);
+  if (rc != ISA_OK) return rc;
+  if (!backward_supported(p))
+    return fail(ISA_ERR_UNSUPPORTED, "the backward pass needs bfloat16 inputs, D = 128 and lengths that b divides");
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv)
+    return fail(ISA_ERR_ARG, "q, k, v, out, lse, dout, dq, dk and dv must not be NULL");
+  const void* in[6] = {q, k, v, out, lse, dout};
+  void* grads[3] = {dq, dk, dv};
+  const size_t io = (size_t)p.BH * p.N * p.D * p.elem;
+  for (int i = 0; i < 6; ++i)
+    if (reinterpret_cast<uintptr_t>(in[i]) & 15) return fail(ISA_ERR_ARG, "every pointer must be 16-byte aligned");
+  for (int g = 0; g < 3; ++g) {
+    if (reinterpret_cast<uintptr_t>(grads[g]) & 15) return fail(ISA_ERR_ARG, "every pointer must be 16-byte aligned");
+    for (int i = 0; i < 6; ++i)
+      if (overlaps2(grads[g], io, in[i], i == 4 ? sizeof(float) * (size_t)p.BH * p.N : io))
+        return fail(ISA_ERR_ARG, "dq, dk and dv must not overlap the inputs");
+    for (int h = 0; h < g; ++h)
+      if (overlaps(grads[g], grads[h], io)) return fail(ISA_ERR_ARG, "dq, dk and dv must not overlap each other");
+  }
+  const size_t need_f = workspace_layout(p, nullptr, nullptr), need_b = backward_workspace_bytes(p);
+  if (!fwd_workspace || fwd_workspace_bytes < need_f)
+    return fail(ISA_ERR_WORKSPACE, "the forward workspace (%zu bytes needed) must be the one of the forward call",
+                need_f);
+  if (!bwd_workspace || bwd_workspace_bytes < need_b)
+    return fail(ISA_ERR_WORKSPACE, "backward workspace too small: %zu bytes given, %zu needed", bwd_workspace_bytes,
+                need_b);
+  if ((reinterpret_cast<uintptr_t>(fwd_workspace) | reinterpret_cast<uintptr_t>(bwd_workspace)) & 255)
+    return fail(ISA_ERR_WORKSPACE, "workspaces must be 256-byte aligned");
+  Work w;
+  workspace_layout(p, &w, static_cast<char*>(fwd_workspace));
+  const cudaError_t e = launch_backward(q, k, v, out, lse, dout, dq, dk, dv, p, w, bwd_workspace,
+                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ISA_OK : cuda_fail(e, "backward launch");
 }
 
 }  // extern "C"

@@ -61,6 +61,8 @@ struct Work {
   float* vct;            // fp32 inputs only: [BH, D, vct_ld] pooled V_new rows transposed
   int32_t* nsel;         // k_ns > 0 only: [BH, n_q, k_ns] exactly computed K_new blocks of each query block, ascending
   uint32_t* nsmask;      // k_ns > 0 only: [BH, n_q, ns_words] the same blocks as a bitmask over K_new's blocks
+  float* lse;            // optional, caller memory (not workspace): [BH, N] per-row log-sum-exp written by the
+                         // attention kernels (training forward); NULL to skip
 };
 
 constexpr int kCtrlWords = 64;
@@ -108,6 +110,15 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
 // by the keys of its exact blocks, in one online softmax.
 cudaError_t launch_attention_ns(const void* q, const void* k, const void* v, void* out, const Plan& p,
                                 const Work& w, cudaStream_t s);
+
+// Backward pass (bf16, D = 128, whole blocks, alpha_ns = 0): whether these sizes are supported,
+// the scratch it needs beyond the forward's workspace, and the launch sequence (delta pass, dQ,
+// dK/dV of the Taylor path over the pooled rows, dK/dV of the exact path plus the Taylor spread).
+bool backward_supported(const Plan& p);
+size_t backward_workspace_bytes(const Plan& p);
+cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                            const void* dout, void* dq, void* dk, void* dv, const Plan& pl, const Work& w,
+                            void* bwd_ws, cudaStream_t s);
 
 // One thread waits on an mbarrier that nothing arrives on; the bounded wait gives
 // up after `timeout_ms` and sets kErrSelftest in err[0].

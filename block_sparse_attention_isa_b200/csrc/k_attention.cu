@@ -107,6 +107,8 @@ struct AttnParams {
   const int32_t* route;
   void* out;
   uint32_t* err;
+  float* lse;          // optional [BH, N] (plain path only): natural log of each row's softmax denominator
+  float taylor_ln_b;   // ln(b): the Taylor rows' weight b, dropped from their exponents, back in their lse
   const uint32_t* nsmask;  // NS: [BH, n_q, ns_words] exact key blocks of every query block
   int ns_words;            // NS: ceil(n_new / 32)
   int npt;                 // NS: K/V tiles of the pooled rows, ceil(n_new / 128)
@@ -769,9 +771,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 8; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[i + c]), __uint_as_float(r[i + 8 + c]));
         }
-        const float mx = fmaxf(fmax3(mc[0], mc[1], mc[2]), fmax3(fmax3(mc[3], mc[4], mc[5]), mc[6], mc[7])) *
-                             p.scale_log2 +
-                         bias;
+        const float raw_max = fmaxf(fmax3(mc[0], mc[1], mc[2]), fmax3(fmax3(mc[3], mc[4], mc[5]), mc[6], mc[7]));
+        const float mx = raw_max * p.scale_log2 + bias;
         // lazy max: move it only when the tile's max exceeds it by more than 2^8
         const bool need = (j > 0) && (mx > m + kRescaleThreshold);
         const float alpha = need ? ex2_approx(m - mx) : 1.0f;
@@ -808,22 +809,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint64_t e;
             if (i % kPolyDen < kPolyNum) e = exp2_poly2(x);
             else e = pack2(ex2_approx(lo2(x)), ex2_approx(hi2(x)));
+            acc[i & 3] = fadd2(acc[i & 3], e);
             if constexpr (sizeof(T) == 2) {
               __nv_bfloat162 hv = __floats2bfloat162_rn(lo2(e), hi2(e));
               r[i] = *reinterpret_cast<uint32_t*>(&hv);
             } else {
-              acc[i & 3] = fadd2(acc[i & 3], e);
               r[2 * i] = static_cast<uint32_t>(e);
               r[2 * i + 1] = static_cast<uint32_t>(e >> 32);
             }
-          }
-          if constexpr (sizeof(T) == 2) {
-            // the row sum adds the same bf16 values that the P V MMA multiplies: with the lazy
-            // maximum the dominant keys' p lie in (1, 2^8] and round in bf16, and a sum of the
-            // unrounded p would leave numerator and denominator up to 2^-9 apart on them
-#pragma unroll
-            for (int i = half * kCols / 4; i < (half + 1) * kCols / 4; ++i)
-              acc[i & 1] = fadd2(acc[i & 1], pack2(__uint_as_float(r[i] << 16), __uint_as_float(r[i] & 0xffff0000u)));
           }
           // this half's P: bf16 pairs in kCols/4 columns, or fp32 in kCols/2 columns
           constexpr int kPCols = sizeof(T) == 2 ? kCols / 4 : kCols / 2;
@@ -837,8 +830,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(&bars->p_half[t][half]);
         }
+        // bf16: the P V MMA multiplies the bf16 p, the row sum takes the fp32 p except that the
+        // tile's largest p enters as its bf16 value. With the lazy maximum a row's dominant keys
+        // have p in (1, 2^8], which bf16 rounds by up to 2^-9: left in the sum, that mismatch
+        // between numerator and denominator would scale the whole output row by it.
+        float corr = 0.f;
+        if constexpr (sizeof(T) == 2) {
+          const float em = ex2_approx(fmaf(raw_max, p.scale_log2, nm));  // the largest p, as computed above
+          corr = __bfloat162float(__float2bfloat16_rn(em)) - em;
+        }
         const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-        l = l * alpha + (lo2(a2) + hi2(a2));
+        l = l * alpha + ((lo2(a2) + hi2(a2)) + corr);
         ++pv_cnt;
       }
       if (!ok) break;
@@ -850,6 +852,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool store = (u < it.nblk) && (row % p.b) < qblock_len(p, qb);  // rows past a short block: none
       const size_t token = (size_t)qblock_start(p, qb) + (row % p.b);
       T* dst = out + ((size_t)it.bh * p.N + token) * D;
+      if (!NS && p.lse && store)  // m and log2(l) are base 2; the weight b is not in the Taylor exponents
+        p.lse[(size_t)it.bh * p.N + token] =
+            (m + __log2f(l)) * 0.6931471805599453f + (it.kind == 1 ? p.taylor_ln_b : 0.f);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -878,6 +883,8 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, void* out, con
   using C = Cfg<T, D>;
   AttnParams p{};
   p.route = w.route;
+  p.lse = NS ? nullptr : w.lse;
+  p.taylor_ln_b = logf((float)pl.b);
   p.out = out;
   p.err = w.ctrl;
   p.BH = pl.BH;

@@ -96,6 +96,8 @@ struct PairParams {
   const int32_t* route;
   void* out;
   uint32_t* err;
+  float* lse;          // optional [BH, N]: natural log of each row's softmax denominator
+  float taylor_ln_b;   // ln(b): the Taylor rows' weight b, dropped from their exponents, back in their lse
   // short blocks: sel [BH, k] kept context blocks (a kept short block is the last one kept)
   const int32_t* sel;
   int k, n_src, L_srcp, len_src_last, len_ctx_last, ragged;
@@ -577,8 +579,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[40 + c]), __uint_as_float(r[48 + c]));
 #pragma unroll
         for (int c = 0; c < 8; ++c) mc[c] = fmaxf(mc[c], __uint_as_float(r[56 + c]));
-        const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7])) *
-                         p.scale_log2;
+        const float raw_max = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+        const float mx = raw_max * p.scale_log2;
         const bool need = (j > 0) && (mx > m + kRescaleThreshold);
         const float alpha = need ? ex2_approx(m - mx) : 1.0f;
         if (j == 0 || need) m = mx;
@@ -594,10 +596,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tmem_st32(t_o + 32 * c, o);
           }
         }
-        // p = 2^(s * scale - m) in pairs, written over this tile's S buffer as bf16 pairs. The row
-        // sum adds the same bf16 values that the P V MMA multiplies: with the lazy maximum, the
-        // dominant keys' p lie in (1, 2^8] and round in bf16, and a sum of the unrounded p would
-        // leave numerator and denominator up to 2^-9 apart on them
+        // The P V MMA multiplies the bf16 p; the row sum takes the fp32 p, except that the tile's
+        // largest p enters as its bf16 value. With the lazy maximum a row's dominant keys have p
+        // in (1, 2^8], which bf16 rounds by up to 2^-9: left in the sum, that mismatch between
+        // numerator and denominator would scale the whole output row by it.
+        const float em = ex2_approx(fmaf(raw_max, p.scale_log2, -m));  // the largest p, as computed below
+        const float corr = __bfloat162float(__float2bfloat16_rn(em)) - em;
+        // p = 2^(s * scale - m) in pairs, written over this tile's S buffer as bf16 pairs
         const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(-m, -m);
         uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -605,17 +610,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint64_t x =
               ffma2(static_cast<uint64_t>(r[2 * i]) | (static_cast<uint64_t>(r[2 * i + 1]) << 32), sc2, nm2);
           const uint64_t e = (i % kPolyDen < kPolyNum) ? exp2_poly2(x) : pack2(ex2_approx(lo2(x)), ex2_approx(hi2(x)));
+          acc[i & 3] = fadd2(acc[i & 3], e);
           __nv_bfloat162 hv = __floats2bfloat162_rn(lo2(e), hi2(e));
-          const uint32_t hb = *reinterpret_cast<uint32_t*>(&hv);
-          r[i] = hb;
-          acc[i & 3] = fadd2(acc[i & 3], pack2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u)));
+          r[i] = *reinterpret_cast<uint32_t*>(&hv);
         }
         tmem_st32(buf, r);
         tmem_st_wait();
         tc_fence_before();
         arrive_cluster(p_full_l + 8u * (seq & 1));
         const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-        l = l * alpha + (lo2(a2) + hi2(a2));
+        l = l * alpha + ((lo2(a2) + hi2(a2)) + corr);
       }
       if (!ok) break;
       // epilogue: O / l at the row's original token position
@@ -627,6 +631,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool store = (ut < it.ntiles) && (u < it.nblk) && (row % p.b) < qblock_len(p, qb);
       const size_t token = (size_t)qblock_start(p, qb) + (row % p.b);
       __nv_bfloat16* dst = out + ((size_t)it.bh * p.N + token) * kD;
+      if (p.lse && store)  // log of the row's denominator: m and log2(l) are base 2 (a short pooled
+                           // row's length is already in its exponent, the weight b is not)
+        p.lse[(size_t)it.bh * p.N + token] =
+            (m + __log2f(l)) * 0.6931471805599453f + (it.kind == 1 ? p.taylor_ln_b : 0.f);
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
         uint32_t o[32];
@@ -677,6 +685,8 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
   p.route = w.route;
   p.out = out;
   p.err = w.ctrl;
+  p.lse = w.lse;
+  p.taylor_ln_b = logf((float)pl.b);
   p.BH = pl.BH;
   p.N = pl.N;
   p.b = pl.b;

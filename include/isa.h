@@ -306,6 +306,49 @@ ISA_API int isa_forward_varlen(const void* q, const void* k, const void* v, int 
                                void* out, int32_t* dbg_sel, int32_t* dbg_route, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/*
+ * Training (trainable ISA: papernotes.org, overview and Key design 2; paperlayer.ai
+ * summary, appendix H, where the kernels implement the forward and the backward
+ * pass). The backward holds the forward's discrete decisions fixed (kept context
+ * blocks and routing): the gradient flows through the exact path over K_new /
+ * V_new, the Taylor path over the block means (a mean spreads its gradient as
+ * 1/b over its block's rows) and the gather (a kept context block's rows get
+ * their K_new rows' gradient; the other context rows get none). The pooling
+ * probe, the top-k and the sharpness carry no gradient.
+ *
+ * isa_forward_train - isa_forward_ex (alpha_ns = 0) that also writes
+ *   lse   device float32 [B, H, N], 16-byte aligned: for every row the natural
+ *         log of its softmax denominator, sum_t exp(q . k_t / sqrt(D)) over
+ *         K_new for an exact row, sum_j L_K(j) exp(q . Kc_j / sqrt(D)) over the
+ *         blocks of K_new for a Taylor row (L_K = the block's length).
+ * The workspace then holds the call's decisions and pooled rows; keep it, unused
+ * by other calls, until isa_backward has run. Debug outputs are not offered.
+ */
+ISA_API int isa_forward_train(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D,
+                              int b, float alpha_s, float alpha_f, isa_dtype dt, void* out, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Scratch that isa_backward needs beyond the forward's workspace (0 if the arguments are invalid). */
+ISA_API size_t isa_backward_workspace_bytes(int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s,
+                                            isa_dtype dt);
+
+/*
+ * isa_backward - gradients of sum(out * dout) with respect to q, k and v, enqueued on
+ * `stream`. Needs bfloat16, D = 128 and lengths that b divides (else
+ * ISA_ERR_UNSUPPORTED). All pointers are device pointers, 16-byte aligned.
+ *   q, k, v, out, lse  the forward call's inputs and outputs (isa_forward_train)
+ *   dout               [B, H, N, D] gradient of the output
+ *   dq, dk, dv         [B, H, N, D] outputs (bfloat16), not overlapping the inputs
+ *   fwd_workspace      the workspace of that isa_forward_train call, untouched since
+ *   bwd_workspace      at least isa_backward_workspace_bytes(), 256-byte aligned
+ * Other arguments must equal the forward call's. Asynchronous, no allocation. A
+ * kernel wait that gives up is reported by isa_device_status(fwd_workspace).
+ */
+ISA_API int isa_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                         const void* dout, int B, int H, int L_src, int L_ctx, int D, int b, float alpha_s,
+                         float alpha_f, isa_dtype dt, void* dq, void* dk, void* dv, void* fwd_workspace,
+                         size_t fwd_workspace_bytes, void* bwd_workspace, size_t bwd_workspace_bytes, void* stream);
+
 /* Message of the last failed call on this host thread ("" if none). */
 ISA_API const char* isa_last_error(void);
 

@@ -97,3 +97,39 @@ def isa_slice_grad_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, dout: np.nda
     out = slice_forward_torch(qt, kt, vt, sr)
     out.backward(torch.tensor(np.asarray(dout, np.float64)))
     return dict(out=out.detach().numpy(), dq=qt.grad.numpy(), dk=kt.grad.numpy(), dv=vt.grad.numpy(), sr=sr)
+
+
+def isa_slice_lse_ref(q: np.ndarray, k: np.ndarray, L_src: int, L_ctx: int, b: int, alpha_s: float,
+                      alpha_f: float, sr: Optional[Dict[str, object]] = None) -> np.ndarray:
+    """Per-row log-sum-exp of the forward's softmax denominators (float64, [N]), alpha_ns = 0.
+
+    The quantity a trainable kernel saves for its backward pass (papernotes.org, overview and
+    "Key design 2": the online softmax keeps a running maximum and sum per row):
+    * an exact-path row q: log sum_t exp(q . K_new_t / sqrt(D)) over every key of K_new;
+    * a Taylor-path row q: log sum_j L_K(j) exp(q . Kc_j / sqrt(D)) over the blocks j of K_new,
+      each weighing its length L_K(j) (b for a whole block), i.e. the log of the literal
+      denominator l of "Key design 2".
+    """
+    if sr is None:
+        sr = R.isa_select_route_ragged(q, k, L_src, L_ctx, b, alpha_s, alpha_f)
+    N, D = q.shape
+    bounds, n_src = sr["bounds"], int(sr["n_src"])
+    new_blocks = list(range(n_src)) + [n_src + int(c) for c in sr["sel"]]
+    rows = [t for j in new_blocks for t in range(*bounds[j])]
+    k_new = np.asarray(k, np.float64)[rows]
+    kc = np.stack([np.asarray(k[s:e], np.float64).mean(axis=0) for s, e in (bounds[j] for j in new_blocks)])
+    ln_len = np.log(np.array([bounds[j][1] - bounds[j][0] for j in new_blocks], np.float64))
+    q64 = np.asarray(q, np.float64)
+    out = np.zeros(N, np.float64)
+
+    def lse(z):
+        m = z.max(axis=1, keepdims=True)
+        return (m + np.log(np.exp(z - m).sum(axis=1, keepdims=True)))[:, 0]
+
+    for i in sr["exact"]:
+        s, e = bounds[int(i)]
+        out[s:e] = lse(q64[s:e] @ k_new.T / math.sqrt(D))
+    for i in sr["taylor"]:
+        s, e = bounds[int(i)]
+        out[s:e] = lse(q64[s:e] @ kc.T / math.sqrt(D) + ln_len[None, :])
+    return out

@@ -261,3 +261,58 @@ def test_varlen_argument_errors(L):
     big = [64] * 5000
     assert L.isa_forward_varlen(FAKE, FAKE, FAKE, 5000, 1, _arr(big), _arr(big), 64, 64, 0.5, 0.5, 0, FAKE, None,
                                 None, None, 0, None) == -3
+
+
+def _bwd(L, B=1, H=2, L_src=512, L_ctx=512, D=128, b=64, dt=0, ptrs=None, fws=None, fws_bytes=0, bws=None,
+         bws_bytes=0):
+    p = ptrs or [FAKE + (i << 32) for i in range(9)]
+    return L.isa_backward(p[0], p[1], p[2], p[3], p[4], p[5], B, H, L_src, L_ctx, D, b, 0.5, 0.5, dt, p[6], p[7],
+                          p[8], fws, fws_bytes, bws, bws_bytes, None)
+
+
+def test_backward_workspace_bytes(L):
+    # delta [BH, N] and dKc, dVc [BH, n_new, D] in float32, each part rounded up to 256 bytes
+    n_new = 8 + 4  # 8 source blocks + ceil(0.5 * 8) kept
+    want = 4 * 2 * 1024 + 2 * 4 * 2 * n_new * 128
+    assert L.isa_backward_workspace_bytes(1, 2, 512, 512, 128, 64, 0.5, 0) == want
+    assert L.isa_backward_workspace_bytes(1, 2, 512, 512, 96, 64, 0.5, 0) == 0
+
+
+@pytest.mark.parametrize("kw,code,msg", [
+    (dict(L_src=500), -3, "b divides"),         # a short last block
+    (dict(D=64), -3, "D = 128"),
+    (dict(dt=1, D=64), -3, "bfloat16"),
+    (dict(), -4, "forward workspace"),           # no forward workspace
+    (dict(fws=FAKE + (10 << 32), fws_bytes=1 << 30), -4, "backward workspace"),
+])
+def test_backward_argument_checks(L, kw, code, msg):
+    assert _bwd(L, **kw) == code
+    assert msg in isa.last_error()
+
+
+def test_backward_pointer_checks(L):
+    p = [FAKE + (i << 32) for i in range(9)]
+    p[5] += 8  # dout misaligned
+    assert _bwd(L, ptrs=p) == -1 and "aligned" in isa.last_error()
+    p = [FAKE + (i << 32) for i in range(9)]
+    p[7] = p[1] + 64  # dk inside k
+    assert _bwd(L, ptrs=p) == -1 and "overlap" in isa.last_error()
+    p = [FAKE + (i << 32) for i in range(9)]
+    p[8] = p[6]  # dv is dq
+    assert _bwd(L, ptrs=p) == -1 and "overlap" in isa.last_error()
+    p = [FAKE + (i << 32) for i in range(9)]
+    p[6] = p[4] + 2 * 1024 * 4  # dq right after lse (its [B, H, N] float32 extent): allowed, fails later on the workspace
+    assert _bwd(L, ptrs=p) == -4
+    p = [FAKE + (i << 32) for i in range(9)]
+    p[3] = None
+    assert _bwd(L, ptrs=p) == -1
+
+
+def test_forward_train_checks(L):
+    def call(lse, ws=None, ws_bytes=0):
+        return L.isa_forward_train(FAKE, FAKE + (1 << 32), FAKE + (2 << 32), 1, 2, 512, 512, 128, 64, 0.5, 0.5, 0,
+                                   FAKE + (3 << 32), lse, ws, ws_bytes, None)
+    assert call(None) == -1 and "lse" in isa.last_error()
+    assert call(FAKE + (4 << 32) + 4) == -1 and "aligned" in isa.last_error()
+    assert call(FAKE + 64) == -1 and "overlap" in isa.last_error()
+    assert call(FAKE + (4 << 32)) == -4  # no workspace

@@ -49,12 +49,13 @@ def test_varlen_batch_parity(case):
     import block_sparse_attention_isa_b200 as isa
     name, H, D, b, a_s, a_f, lens = case
     parts = [_element(H, D, b, a_s, a_f, ls, lc, i) for i, (ls, lc) in enumerate(lens)]
-    flat = [np.concatenate([p[j].ravel() for p in parts]) for j in range(3)]
+    # the packed batch as [total rows, D]: the binding takes D from the last dimension
+    flat = [np.concatenate([p[j].reshape(-1, D) for p in parts]) for j in range(3)]
     tq, tk, tv = (torch.from_numpy(x).to("cuda", torch.bfloat16) for x in flat)
     Ls, Lc = [ls for ls, _ in lens], [lc for _, lc in lens]
     out, sel, route = isa.forward_varlen(tq, tk, tv, H, Ls, Lc, b, a_s, a_f, debug=True)
     isa.device_status()
-    out, sel, route = out.float().cpu().numpy(), sel.cpu().numpy(), route.cpu().numpy()
+    out, sel, route = out.float().cpu().numpy().ravel(), sel.cpu().numpy(), route.cpu().numpy()
     off = off_s = off_r = 0
     for (ls, lc), (_, _, _, refs) in zip(lens, parts):
         N = ls + lc
@@ -77,16 +78,16 @@ def test_varlen_equals_separate_calls():
     H, D, b, a_s, a_f = 2, 128, 128, 0.25, 0.5
     lens = [(1000, 1100), (2048, 2048)]
     parts = [_element(H, D, b, a_s, a_f, ls, lc, i) for i, (ls, lc) in enumerate(lens)]
-    flat = [np.concatenate([p[j].ravel() for p in parts]) for j in range(3)]
+    flat = [np.concatenate([p[j].reshape(-1, D) for p in parts]) for j in range(3)]
     tq, tk, tv = (torch.from_numpy(x).to("cuda", torch.bfloat16) for x in flat)
     out = isa.forward_varlen(tq, tk, tv, H, [l[0] for l in lens], [l[1] for l in lens], b, a_s, a_f)
     isa.device_status()
     off = 0
     for (ls, lc) in lens:
-        n = H * (ls + lc) * D
+        n = H * (ls + lc)
         shp = (1, H, ls + lc, D)
         one = isa.forward(tq[off:off + n].view(shp), tk[off:off + n].view(shp), tv[off:off + n].view(shp), ls, lc,
                           b, a_s, a_f)
         isa.device_status()
-        assert torch.equal(one.view(-1), out[off:off + n])
+        assert torch.equal(one.view(-1, D), out[off:off + n])
         off += n

@@ -106,3 +106,61 @@ def test_taylor_only_gradients_are_constant_inside_blocks():
             else:
                 np.testing.assert_allclose(grad[s:e], np.broadcast_to(grad[s], grad[s:e].shape), rtol=1e-12,
                                            atol=1e-15)
+
+
+# ----------------------------------------------------------------------------- per-row log-sum-exp
+
+def test_lse_at_dense_point_is_torch_logsumexp():
+    """alpha_s = 1, alpha_f = 0: every row is exact over all keys, so the saved statistic is the
+    log-sum-exp of q K^T / sqrt(D) (a library routine)."""
+    import isa_synth
+    from oracle import isa_oracle_backward as BW
+    w = isa_synth.Workload("t", 1, 1, 16, 48, 40, 8, 1.0, 0.0, 0.1, 1.0, 0.5, "f32")
+    q, k, _ = isa_synth.make_slice(w, 2, 0, 0, 0)
+    got = BW.isa_slice_lse_ref(q, k, w.L_src, w.L_ctx, w.b, 1.0, 0.0)
+    tq, tk = torch.from_numpy(q.astype(np.float64)), torch.from_numpy(k.astype(np.float64))
+    want = torch.logsumexp(tq @ tk.T / math.sqrt(16), dim=1).numpy()
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("L_src,L_ctx,a_s,a_f", [(64, 64, 0.5, 0.5), (61, 70, 0.5, 0.75), (64, 48, 1.0, 1.0)])
+def test_lse_reproduces_the_forward_output(L_src, L_ctx, a_s, a_f):
+    """exp(logit - lse) are the normalised weights: with them each row's weighted sum of its
+    values is the forward output (exact rows over V_new, Taylor rows over the block means with
+    the length weight), also with short last blocks."""
+    import isa_synth
+    from oracle import isa_oracle_backward as BW
+    from oracle import isa_oracle_ragged as RR
+    b, D = 8, 16
+    w = isa_synth.Workload("t", 1, 1, D, L_src, L_ctx, b, a_s, a_f, 0.1, 1.0, 0.5, "f32")
+    q, k, v = isa_synth.make_slice(w, 4, 0, 0, 0)
+    sr = RR.isa_select_route_ragged(q, k, L_src, L_ctx, b, a_s, a_f)
+    ref = RR.isa_slice_ref_ragged(q, k, v, L_src, L_ctx, b, a_s, a_f, sr=sr)
+    lse = BW.isa_slice_lse_ref(q, k, L_src, L_ctx, b, a_s, a_f, sr=sr)
+    bounds, new_b = ref["bounds"], ref["new_bounds"]
+    k_new, v_new = ref["k_new"], ref["v_new"]
+    for i in sr["exact"]:
+        s, e = bounds[int(i)]
+        p = np.exp(q[s:e].astype(np.float64) @ k_new.T / math.sqrt(D) - lse[s:e, None])
+        np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-12)
+        np.testing.assert_allclose(p @ v_new, ref["out"][s:e], atol=1e-12)
+    kc = np.stack([k_new[a:z].mean(axis=0) for a, z in new_b])
+    vc = np.stack([v_new[a:z].mean(axis=0) for a, z in new_b])
+    ln = np.log([z - a for a, z in new_b])
+    for i in sr["taylor"]:
+        s, e = bounds[int(i)]
+        p = np.exp(q[s:e].astype(np.float64) @ kc.T / math.sqrt(D) + ln[None, :] - lse[s:e, None])
+        np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-12)
+        np.testing.assert_allclose(p @ vc, ref["out"][s:e], atol=1e-12)
+
+
+def test_lse_taylor_with_block_size_one_is_dense():
+    """b = 1: pooling is the identity and every weight is 1, so a Taylor row's statistic is the
+    dense log-sum-exp."""
+    import isa_synth
+    from oracle import isa_oracle_backward as BW
+    w = isa_synth.Workload("t", 1, 1, 8, 20, 12, 1, 1.0, 1.0, 0.1, 1.0, 0.5, "f32")
+    q, k, _ = isa_synth.make_slice(w, 6, 0, 0, 0)
+    got = BW.isa_slice_lse_ref(q, k, 20, 12, 1, 1.0, 1.0)
+    tq, tk = torch.from_numpy(q.astype(np.float64)), torch.from_numpy(k.astype(np.float64))
+    np.testing.assert_allclose(got, torch.logsumexp(tq @ tk.T / math.sqrt(8), dim=1).numpy(), atol=1e-12)
