@@ -502,6 +502,63 @@ def run_ours(args, w):
         dist.destroy_process_group()
 
 
+def backward_flops_per_call(w) -> dict:
+    """FLOPs of the backward pass: algorithmic = the five products per path (S and dP recomputed,
+    dV, dK, dQ), each 2 * rows * keys * D; executed = the seven the two kernels issue (S and dP are
+    computed once in the dQ kernel and once, transposed, in the dK/dV kernel)."""
+    n_src, n_ctx = _cdiv(w.L_src, w.b), _cdiv(w.L_ctx, w.b)
+    n_q = n_src + n_ctx
+    k = max(0, min(n_ctx, math.ceil(float(np.float32(w.alpha_s)) * n_ctx - 1e-4)))
+    n_flat = max(0, min(n_q, math.floor(float(np.float32(w.alpha_f)) * n_q + 1e-4)))
+    n_new = n_src + k
+    bh = w.B * w.H
+    unit = 2.0 * w.D * bh * w.b * ((n_q - n_flat) * n_new * w.b + n_flat * n_new)
+    return {"algorithmic": 5.0 * unit, "executed": 7.0 * unit}
+
+
+def run_backward(args, w):
+    """Time the backward pass (isa_backward, after one training forward) at this workload."""
+    import torch
+    import block_sparse_attention_isa_b200 as isa
+    from block_sparse_attention_isa_b200 import build as isa_build
+    torch.cuda.set_device(0)
+    isa_build.build()
+    dev = torch.device("cuda", 0)
+    q, k, v = workload_inputs(w, full=getattr(args, "full_workload", None))
+    tq, tk, tv = (torch.from_numpy(x).to(dev, torch.bfloat16) for x in (q, k, v))
+    g = torch.randn(tq.shape, generator=torch.Generator().manual_seed(5)).to(dev, torch.bfloat16)
+    out, lse, ws = isa.forward_train(tq, tk, tv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f)
+    nb = isa.lib().isa_backward_workspace_bytes(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, 0)
+    bws = torch.empty(nb, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        isa.backward(tq, tk, tv, out, lse, g, ws, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, bwd_workspace=bws)
+    isa.device_status(ws)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    start.record()
+    for _ in range(args.steps):
+        isa.backward(tq, tk, tv, out, lse, g, ws, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, bwd_workspace=bws)
+    end.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    isa.device_status(ws)
+    ms = start.elapsed_time(end) / args.steps
+    f = backward_flops_per_call(w)
+    peaks, kind = load_peaks()
+    peak, which = roofline_peak(peaks, args.steps * ms * 1e-3)
+    line = {"metric": "ISA backward ms/call and TFLOPS", "value": f["algorithmic"] / (ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
+            "config": {"workload": workload_label(args, w), "B": w.B, "H": w.H, "N": w.N, "D": w.D, "b": w.b,
+                       "alpha_s": w.alpha_s, "alpha_f": w.alpha_f},
+            "flops": f, "executed_tflops": f["executed"] / (ms * 1e-3) / 1e12,
+            "frac_algorithmic": f["algorithmic"] / (ms * 1e-3) / 1e12 / peak,
+            "frac_executed": f["executed"] / (ms * 1e-3) / 1e12 / peak,
+            "peak": peak, "peak_kind": f"{kind} bf16 {which}", "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -517,6 +574,8 @@ def main():
     ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
                     help="N > 1: weak = one batch element per rank; strong = the workload's heads split over ranks")
     ap.add_argument("--gather", action="store_true", help="strong scaling: all-gather O over NCCL in every step")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (training) instead of the forward; one GPU, not a bench line")
     ap.add_argument("--heads", type=int, default=0,
                     help="run only the first H heads of the workload (small profiling captures; not a bench line)")
     args = ap.parse_args()
@@ -526,7 +585,9 @@ def main():
         args.full_workload = w
         w = w.with_(H=min(args.heads, w.H))
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
-    if args.impl == "reference":
+    if args.backward:
+        run_backward(args, w)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_ours(args, w)

@@ -47,6 +47,8 @@ def up_to_date() -> bool:
 REGISTER_SPLIT_KERNELS = {
     "attention_pair_kernel": 168,
     "attention_kernel": 168,
+    "attention_mixed_kernel": 168,
+    "attention_bwd_kernel": 168,
 }
 
 

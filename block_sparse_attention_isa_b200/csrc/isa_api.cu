@@ -232,8 +232,11 @@ int run_forward(const void* q, const void* k, const void* v, const Plan& p, void
     e = use_pair_kernel(pe) ? launch_attention_pair(q, k, v, out, pe, w, s, nullptr)
                                      : launch_attention(q, k, v, out, pe, w, s, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-    if (p.k_ns > 0 && p.n_flat > 0 && (e = launch_attention_ns(q, k, v, out, p, w, s)) != cudaSuccess)
-      return cuda_fail(e, "mixed Taylor attention launch");
+    if (p.k_ns > 0 && p.n_flat > 0) {
+      e = attention_mixed_supported(p) ? launch_attention_mixed(q, k, v, out, p, w, s)
+                                       : launch_attention_ns(q, k, v, out, p, w, s);
+      if (e != cudaSuccess) return cuda_fail(e, "mixed Taylor attention launch");
+    }
   }
   if ((e = mark(4, s)) != cudaSuccess) return cuda_fail(e, "recording a stage event");
   if (dbg_sel && p.k > 0) {

@@ -110,6 +110,11 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
 // by the keys of its exact blocks, in one online softmax.
 cudaError_t launch_attention_ns(const void* q, const void* k, const void* v, void* out, const Plan& p,
                                 const Work& w, cudaStream_t s);
+// The same for bf16, D = 128, b = 128 and whole blocks: one query block per work item, the two
+// softmax warpgroups on alternate key tiles of it, their softmax states merged at the end.
+bool attention_mixed_supported(const Plan& p);
+cudaError_t launch_attention_mixed(const void* q, const void* k, const void* v, void* out, const Plan& p,
+                                   const Work& w, cudaStream_t s);
 
 // Backward pass (bf16, D = 128, whole blocks, alpha_ns = 0): whether these sizes are supported,
 // the scratch it needs beyond the forward's workspace, and the launch sequence (delta pass, dQ,

@@ -831,13 +831,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&bars->p_half[t][half]);
         }
         // bf16: the P V MMA multiplies the bf16 p, the row sum takes the fp32 p except that the
-        // tile's largest p enters as its bf16 value. With the lazy maximum a row's dominant keys
-        // have p in (1, 2^8], which bf16 rounds by up to 2^-9: left in the sum, that mismatch
-        // between numerator and denominator would scale the whole output row by it.
+        // tile's largest p enters as its bf16 value when it exceeds 1. With the lazy maximum a
+        // row's dominant keys have p in (1, 2^8] (only in tiles whose maximum exceeds m), which
+        // bf16 rounds by up to 2^-9: left in the sum, that mismatch between numerator and
+        // denominator would scale the whole output row by it. (A key that set m has p = 1.)
         float corr = 0.f;
         if constexpr (sizeof(T) == 2) {
-          const float em = ex2_approx(fmaf(raw_max, p.scale_log2, nm));  // the largest p, as computed above
-          corr = __bfloat162float(__float2bfloat16_rn(em)) - em;
+          if (mx > m) {
+            const float em = ex2_approx(fmaf(raw_max, p.scale_log2, nm));  // the largest p, as computed above
+            corr = __bfloat162float(__float2bfloat16_rn(em)) - em;
+          }
         }
         const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
         l = l * alpha + ((lo2(a2) + hi2(a2)) + corr);

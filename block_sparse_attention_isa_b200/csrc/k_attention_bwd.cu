@@ -32,9 +32,11 @@
 // accumulating MMAs take P / dS from TMEM and the column tile as an MN-major B.
 // TMEM: S and T double-buffered (columns [0,128) and [128,256)), accumulators at
 // [256, 384) (dV or dQ) and [384, 512) (dK). Warp 0 issues the TMA loads, warp 1
-// the MMAs (one thread), warps 4-7 are the elementwise warpgroup. While the
-// warpgroup works on column tile j, the tensor core computes S and T of tile
-// j + 1; the accumulating MMAs of tile j follow once its P and dS are written.
+// the MMAs (one thread), warps 4-7 and 8-11 are two elementwise warpgroups that
+// take alternate column tiles (one S/T buffer each), so that two tiles' chains
+// of TMEM loads, exponentials and TMEM stores are in flight at once; while they
+// work, the tensor core computes the next tiles' S and T and the accumulating
+// MMAs of the tiles already done.
 // Every wait is bounded; a timeout sets the workspace error word and stops the CTA.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -48,7 +50,13 @@
 namespace isa {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 4-7 and 8-11 the two elementwise warpgroups
+// Register split: warpgroup 0 (TMA, MMA) gives registers back, the elementwise warpgroups take them
+// (384 x 168 at launch = 128 x 88 + 256 x 208).
+constexpr int kLaunchRegs = 168;
+constexpr int kLowRegs = 88;
+constexpr int kHighRegs = 208;
+static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
 constexpr int kD = 128;
 constexpr int kBM = 128;                 // rows of an item
 constexpr int kBN = 64;                  // columns of a tile
@@ -210,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->p_full[b], 128);
     }
     mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->acc_empty, 128);
+    mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     mbar_fence_init();
@@ -232,6 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+
+  if (warp < 4) regs_dealloc<kLowRegs>();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -402,6 +412,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ elementwise + epilogue
+    // Warpgroup w takes the column tiles in S/T buffer w (tiles ct with ct % 2 == w), so the two
+    // work on consecutive tiles at once; both then write half of the item's epilogue.
+    regs_alloc<kHighRegs>();
+    const int w = (warp - 4) >> 2;
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
     const int wl = warp & 3;
     const int row = wl * 32 + lane;
@@ -428,6 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ncols_valid = kDKDV ? 0 : (it.kind == 0 ? p.L_new : p.n_new);
       for (int jj = 0; jj < nc; ++jj, ++ct, ++tile_it) {
         const uint32_t bf = ct & 1;
+        if ((int)bf != w) continue;  // the other warpgroup's tile
         if (!warp_wait(bars, &bars->s_full[bf], (ct >> 1) & 1, p.err)) { ok = false; break; }
         uint32_t s[kBN], t[kBN];
         tmem_ld32(t_s + bf * kBN, s);
@@ -441,16 +456,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float* stat = reinterpret_cast<const float*>(sB + (tile_it % kStages) * kStageBytes + 2 * kBTile);
           // columns are queries: P^T = 2^(S^T c - lse2_col), dS^T = P^T (T^T - delta_col)
 #pragma unroll
-          for (int i = 0; i < kBN / 2; ++i) {
-            const float2 l2 = *reinterpret_cast<const float2*>(stat + 2 * i);
-            const float2 de = *reinterpret_cast<const float2*>(stat + kBN + 2 * i);
-            const uint64_t nl = pack2(path_off - l2.x * kLog2e, path_off - l2.y * kLog2e);
-            const uint64_t x = ffma2(pack2(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nl);
-            const float e0 = ex2_approx(lo2(x)), e1 = ex2_approx(hi2(x));
-            const uint64_t ds = fmul2(pack2(e0, e1), fadd2(pack2(__uint_as_float(t[2 * i]), __uint_as_float(t[2 * i + 1])),
-                                                            pack2(-de.x, -de.y)));
-            pw[i] = bf16x2(e0, e1);
-            dw[i] = bf16x2(lo2(ds), hi2(ds));
+          for (int i = 0; i < kBN / 2; i += 2) {
+            const float4 l4 = *reinterpret_cast<const float4*>(stat + 2 * i);
+            const float4 d4 = *reinterpret_cast<const float4*>(stat + kBN + 2 * i);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int ii = i + h;
+              const float la = h ? l4.z : l4.x, lb = h ? l4.w : l4.y;
+              const float da = h ? d4.z : d4.x, db = h ? d4.w : d4.y;
+              const uint64_t nl = pack2(path_off - la * kLog2e, path_off - lb * kLog2e);
+              const uint64_t x = ffma2(pack2(__uint_as_float(s[2 * ii]), __uint_as_float(s[2 * ii + 1])), sc2, nl);
+              const float e0 = ex2_approx(lo2(x)), e1 = ex2_approx(hi2(x));
+              const uint64_t ds = fmul2(pack2(e0, e1), fadd2(pack2(__uint_as_float(t[2 * ii]),
+                                                                    __uint_as_float(t[2 * ii + 1])),
+                                                              pack2(-da, -db)));
+              pw[ii] = bf16x2(e0, e1);
+              dw[ii] = bf16x2(lo2(ds), hi2(ds));
+            }
           }
         } else {
           // columns are keys: P = 2^(S c - lse2_row), dS = P (T - delta_row); keys past the end are 0
@@ -486,24 +508,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (kDKDV) {
         const int r = it.row0 + row;  // row of K_new (exact) or pooled row (Taylor)
         const bool valid = row < it.rows;
+        // warpgroup 0 writes dV (accumulator 0), warpgroup 1 dK (accumulator 1, times 1/sqrt(D))
+        const uint32_t t_acc = w == 0 ? t_acc0 : t_acc1;
+        const float scl = w == 0 ? 1.0f : p.inv_sqrt_d;
         if (it.kind == 1) {
           // Taylor: add this column range's partial dKc / dVc (several chunks share a row tile)
           if (nc == 0) continue;  // (not reached: every chunk holds a column tile)
-          float* dkc = p.dkc + ((size_t)it.bh * p.n_new + r) * kD;
-          float* dvc = p.dvc + ((size_t)it.bh * p.n_new + r) * kD;
+          float* dst = (w == 0 ? p.dvc : p.dkc) + ((size_t)it.bh * p.n_new + r) * kD;
 #pragma unroll 1
           for (int c = 0; c < kD / 32; ++c) {
-            uint32_t a0[32], a1[32];
-            tmem_ld32(t_acc0 + 32 * c, a0);
-            tmem_ld32(t_acc1 + 32 * c, a1);
-            tmem_ld_wait<32>(a0);
-            tmem_ld_wait<32>(a1);
+            uint32_t a[32];
+            tmem_ld32(t_acc + 32 * c, a);
+            tmem_ld_wait<32>(a);
             if (valid) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                atomicAdd(dvc + 32 * c + i, __uint_as_float(a0[i]));
-                atomicAdd(dkc + 32 * c + i, __uint_as_float(a1[i]) * p.inv_sqrt_d);
-              }
+              for (int i = 0; i < 32; ++i) atomicAdd(dst + 32 * c + i, __uint_as_float(a[i]) * scl);
             }
           }
         } else {
@@ -519,38 +538,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int blk = r / p.b;
           const float inv_b = 1.0f / (float)p.b;
-          const float* dkc = p.dkc ? p.dkc + ((size_t)it.bh * p.n_new + blk) * kD : nullptr;
-          const float* dvc = p.dvc ? p.dvc + ((size_t)it.bh * p.n_new + blk) * kD : nullptr;
-          __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + ((size_t)it.bh * p.N + (tok < 0 ? 0 : tok)) * kD;
-          __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + ((size_t)it.bh * p.N + (tok < 0 ? 0 : tok)) * kD;
+          const float* spread = (w == 0 ? p.dvc : p.dkc);
+          if (spread) spread += ((size_t)it.bh * p.n_new + blk) * kD;
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(w == 0 ? p.dv : p.dk) +
+                               ((size_t)it.bh * p.N + (tok < 0 ? 0 : tok)) * kD;
 #pragma unroll 1
           for (int c = 0; c < kD / 32; ++c) {
-            float fk[32], fv[32];
+            float f[32];
             if (nc > 0) {
-              uint32_t a0[32], a1[32];
-              tmem_ld32(t_acc0 + 32 * c, a0);
-              tmem_ld32(t_acc1 + 32 * c, a1);
-              tmem_ld_wait<32>(a0);
-              tmem_ld_wait<32>(a1);
+              uint32_t a[32];
+              tmem_ld32(t_acc + 32 * c, a);
+              tmem_ld_wait<32>(a);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                fv[i] = __uint_as_float(a0[i]);
-                fk[i] = __uint_as_float(a1[i]) * p.inv_sqrt_d;
-              }
+              for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(a[i]) * scl;
             } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) fv[i] = fk[i] = 0.f;
+              for (int i = 0; i < 32; ++i) f[i] = 0.f;
             }
             if (tok >= 0) {
-              if (dkc) {
+              if (spread) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                  fk[i] += __ldg(dkc + 32 * c + i) * inv_b;
-                  fv[i] += __ldg(dvc + 32 * c + i) * inv_b;
-                }
+                for (int i = 0; i < 32; ++i) f[i] += __ldg(spread + 32 * c + i) * inv_b;
               }
-              store_bf16_32(dk + 32 * c, fk);
-              store_bf16_32(dv + 32 * c, fv);
+              store_bf16_32(dst + 32 * c, f);
             }
           }
         }
@@ -558,8 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dQ: the row's gradient at its token (rows past the item's last block are copies)
         const bool valid = row < it.rows;
         __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(p.dq) + ((size_t)it.bh * p.N + tok_row) * kD;
+        // warpgroup w writes columns [64 w, 64 w + 64)
 #pragma unroll 1
-        for (int c = 0; c < kD / 32; ++c) {
+        for (int c = 2 * w; c < 2 * w + 2; ++c) {
           uint32_t a0[32];
           tmem_ld32(t_acc0 + 32 * c, a0);
           tmem_ld_wait<32>(a0);
@@ -623,7 +634,11 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* 
                   make_map(&tvc, w.vcn, 2, kD, pl.n_new, pl.BH, 64);
   if (!ok) return cudaErrorInvalidValue;
   auto kern = attention_bwd_kernel<kDKDV>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;  // the register split needs this count
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (e != cudaSuccess) return e;
   int grid = device_sm_count();
   if (grid > p.total) grid = p.total;

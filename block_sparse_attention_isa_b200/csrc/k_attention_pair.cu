@@ -92,14 +92,14 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr int kPolyNum = ISA_PAIR_POLY_NUM;
 constexpr int kPolyDen = ISA_PAIR_POLY_DEN;
 
+// Scalars and the pointers every call uses. (The two pointers that only some instances read travel
+// in PairExtra: with them in this struct, ptxas spilled registers in every instance.)
 struct PairParams {
   const int32_t* route;
   void* out;
   uint32_t* err;
-  float* lse;          // optional [BH, N]: natural log of each row's softmax denominator
   float taylor_ln_b;   // ln(b): the Taylor rows' weight b, dropped from their exponents, back in their lse
-  // short blocks: sel [BH, k] kept context blocks (a kept short block is the last one kept)
-  const int32_t* sel;
+  // short blocks (a kept short block is the last one kept)
   int k, n_src, L_srcp, len_src_last, len_ctx_last, ragged;
   float src_last_bias, ctx_last_bias;  // log2(len / b) / scale_log2: raw-score offsets of short pooled rows
   int BH, N, b, L_src, n_q, n_exact, n_flat, L_new, n_new;
@@ -109,6 +109,11 @@ struct PairParams {
   int items_t;  // Taylor items per head
   int total;    // all items
   float scale_log2;
+};
+
+struct PairExtra {
+  float* lse;          // kLse: [BH, N] natural log of each row's softmax denominator
+  const int32_t* sel;  // kRagged: [BH, k] kept context blocks
 };
 
 struct Bars {
@@ -211,8 +216,8 @@ __device__ __forceinline__ int qblock_len(const PairParams& p, int i) {
   return i == p.n_src - 1 ? p.len_src_last : (i == p.n_q - 1 ? p.len_ctx_last : p.b);
 }
 // Whether head bh keeps the short last context block, which is then the last block of K_new.
-__device__ __forceinline__ bool short_ctx_kept(const PairParams& p, int bh) {
-  return p.len_ctx_last < p.b && p.k > 0 && __ldg(p.sel + (size_t)bh * p.k + p.k - 1) == p.n_q - p.n_src - 1;
+__device__ __forceinline__ bool short_ctx_kept(const PairParams& p, const int32_t* sel, int bh) {
+  return p.len_ctx_last < p.b && p.k > 0 && __ldg(sel + (size_t)bh * p.k + p.k - 1) == p.n_q - p.n_src - 1;
 }
 // -inf for the key rows [lo, hi) of the 64-key tile starting at row `base` (uniform per tile).
 __device__ __forceinline__ void mask_key_rows(uint32_t (&r)[kCols], int base, int lo, int hi) {
@@ -292,11 +297,15 @@ __device__ __forceinline__ void store_row_chunk(__nv_bfloat16* dst, const float*
   for (int i = 0; i < 4; ++i) d[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
 }
 
+// kRagged: the call has a short last block (block starts, masks, length weights); kLse: write each
+// row's lse. Whole-block calls without lse run code with neither.
+template <bool kRagged, bool kLse>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attention_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_ksel, const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_vsel, const __grid_constant__ CUtensorMap tm_kcn,
-                          const __grid_constant__ CUtensorMap tm_vcn, const PairParams p) {
+                          const __grid_constant__ CUtensorMap tm_vcn, const PairParams p,
+                          const PairExtra x) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kOffQ;
@@ -373,7 +382,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int r = 64 * h;
             int u = ut * p.bpt + r / p.b;
             if (u >= it.nblk) u = ut * p.bpt;  // missing block of a partial tile: rows are not stored
-            const int y = qblock_start(p, it.blk(u)) + (r % p.b);  // rows past a short block: not stored
+            // rows past a short block: loaded, not stored
+            const int y = (kRagged ? qblock_start(p, it.blk(u)) : it.blk(u) * p.b) + (r % p.b);
 #pragma unroll
             for (int c = 0; c < 2; ++c)
               tma_load_pair(sQ + t * kQTile + c * kQCh + h * 8192, &tm_q, q_full_l + 8u * t, c * 64, y, it.bh);
@@ -542,7 +552,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int k = 0, g = schedule(p, pair, npairs, 0); g >= 0 && ok; g = schedule(p, pair, npairs, ++k)) {
       const Item it = decode_item(p, g);
       if (t >= it.nslots) continue;
-      const bool cs = p.ragged ? short_ctx_kept(p, it.bh) : false;
+      const bool cs = kRagged ? short_ctx_kept(p, x.sel, it.bh) : false;
       float m = -FLT_MAX, l = 0.f;
       for (int j = 0; j < it.nkv; ++j, ++seq) {
         const uint32_t buf = t_s + (seq & 1) * kBN;
@@ -556,7 +566,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int i = 0; i < kCols; ++i)
             if (i >= it.last_valid) r[i] = __float_as_uint(-INFINITY);
         }
-        if (p.ragged) {  // (uniform branch; the first tile always holds a key of block 0)
+        if constexpr (kRagged) {  // (the first tile always holds a key of block 0)
           if (it.kind == 0) {
             // exact path: the padding rows of the short source block and of a kept short
             // context block (the last block of K_new)
@@ -597,11 +607,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         // The P V MMA multiplies the bf16 p; the row sum takes the fp32 p, except that the tile's
-        // largest p enters as its bf16 value. With the lazy maximum a row's dominant keys have p
-        // in (1, 2^8], which bf16 rounds by up to 2^-9: left in the sum, that mismatch between
-        // numerator and denominator would scale the whole output row by it.
-        const float em = ex2_approx(fmaf(raw_max, p.scale_log2, -m));  // the largest p, as computed below
-        const float corr = __bfloat162float(__float2bfloat16_rn(em)) - em;
+        // largest p enters as its bf16 value when it exceeds 1. With the lazy maximum a row's
+        // dominant keys have p in (1, 2^8] (only in tiles whose maximum exceeds m), which bf16
+        // rounds by up to 2^-9: left in the sum, that mismatch between numerator and denominator
+        // would scale the whole output row by it. (A key that set m has p = 1 exactly.)
+        float corr = 0.f;
+        if (mx > m) {
+          const float em = ex2_approx(fmaf(raw_max, p.scale_log2, -m));  // the largest p, as computed below
+          corr = __bfloat162float(__float2bfloat16_rn(em)) - em;
+        }
         // p = 2^(s * scale - m) in pairs, written over this tile's S buffer as bf16 pairs
         const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(-m, -m);
         uint64_t acc[4] = {0, 0, 0, 0};
@@ -628,13 +642,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int ut = 2 * t + (int)rank;
       const int u = ut * p.bpt + row / p.b;
       const int qb = it.blk((ut < it.ntiles && u < it.nblk) ? u : 0);
-      const bool store = (ut < it.ntiles) && (u < it.nblk) && (row % p.b) < qblock_len(p, qb);
-      const size_t token = (size_t)qblock_start(p, qb) + (row % p.b);
+      const bool store = (ut < it.ntiles) && (u < it.nblk) && (!kRagged || (row % p.b) < qblock_len(p, qb));
+      const size_t token = (size_t)(kRagged ? qblock_start(p, qb) : qb * p.b) + (row % p.b);
       __nv_bfloat16* dst = out + ((size_t)it.bh * p.N + token) * kD;
-      if (p.lse && store)  // log of the row's denominator: m and log2(l) are base 2 (a short pooled
-                           // row's length is already in its exponent, the weight b is not)
-        p.lse[(size_t)it.bh * p.N + token] =
-            (m + __log2f(l)) * 0.6931471805599453f + (it.kind == 1 ? p.taylor_ln_b : 0.f);
+      if constexpr (kLse) {
+        // log of the row's denominator: m and log2(l) are base 2 (a short pooled row's length is
+        // already in its exponent, the weight b is not)
+        if (store)
+          x.lse[(size_t)it.bh * p.N + token] =
+              (m + __log2f(l)) * 0.6931471805599453f + (it.kind == 1 ? p.taylor_ln_b : 0.f);
+      }
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
         uint32_t o[32];
@@ -671,8 +688,13 @@ bool attention_pair_regs_ok() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!cached[dev]) {
     cudaFuncAttributes fa;
-    cached[dev] = (cudaFuncGetAttributes(&fa, attention_pair_kernel) == cudaSuccess && fa.numRegs == kLaunchRegs)
-                      ? 1 : 2;
+    bool ok = true;
+    const void* kernels[4] = {(const void*)attention_pair_kernel<false, false>,
+                              (const void*)attention_pair_kernel<false, true>,
+                              (const void*)attention_pair_kernel<true, false>,
+                              (const void*)attention_pair_kernel<true, true>};
+    for (const void* k : kernels) ok = ok && cudaFuncGetAttributes(&fa, k) == cudaSuccess && fa.numRegs == kLaunchRegs;
+    cached[dev] = ok ? 1 : 2;
   }
   return cached[dev] == 1;
 }
@@ -685,7 +707,6 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
   p.route = w.route;
   p.out = out;
   p.err = w.ctrl;
-  p.lse = w.lse;
   p.taylor_ln_b = logf((float)pl.b);
   p.BH = pl.BH;
   p.N = pl.N;
@@ -696,7 +717,6 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
   p.n_flat = pl.n_flat;
   p.L_new = pl.L_new;
   p.n_new = pl.n_new;
-  p.sel = w.sel;
   p.k = pl.k;
   p.n_src = pl.n_src;
   p.L_srcp = pl.L_srcp;
@@ -725,7 +745,8 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
                   make_map(&tvc, w.vcn, 2, kD, pl.n_new, pl.BH, kBN);
   if (!ok) return cudaErrorInvalidValue;
 
-  auto kern = attention_pair_kernel;
+  auto kern = pl.ragged ? (w.lse ? attention_pair_kernel<true, true> : attention_pair_kernel<true, false>)
+                        : (w.lse ? attention_pair_kernel<false, true> : attention_pair_kernel<false, false>);
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
@@ -733,7 +754,7 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (e != cudaSuccess) return e;
   // as many CTA pairs as can be resident at once (one CTA per SM), at most one per work item
-  static int cached_pairs[64] = {0};
+  static int cached_pairs[64] = {0};  // the same for every instance (same block, shared memory, cluster)
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   int pairs = dev >= 0 && dev < 64 ? cached_pairs[dev] : 0;
@@ -754,7 +775,7 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
     if (dev >= 0 && dev < 64) cached_pairs[dev] = pairs;
   }
   if (pairs > p.total) pairs = p.total;
-  kern<<<2 * pairs, kThreads, kSmemAlloc, s>>>(tq, tk, tks, tv, tvs, tkc, tvc, p);
+  kern<<<2 * pairs, kThreads, kSmemAlloc, s>>>(tq, tk, tks, tv, tvs, tkc, tvc, p, PairExtra{w.lse, w.sel});
   if (n_ctas) *n_ctas = 2 * pairs;
   return cudaGetLastError();
 }
