@@ -40,6 +40,10 @@
 namespace isa {
 namespace {
 
+// Up to this many context blocks the top-k splits by counted ranks (n comparisons per block),
+// above it by a bitonic sort.
+constexpr int kRankSplitMax = 512;
+
 // 16-byte global -> shared copies that complete asynchronously (groups committed and awaited).
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
@@ -322,8 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1) pool_score_topk_kernel(const T* _
         sidx[c] = 0x7fffffff - (c - n_ctx);
       }
     }
-    bitonic_sort_pairs<true>(skey, sidx, P);
     const int kk = p.k;
+    if (n_ctx <= kRankSplitMax) {
+      // the kk best context blocks by counted ranks (ties to the lower index), ascending
+      rank_split<true>(skey, n_ctx, kk, sidx, w.sel + (size_t)bh * kk, nullptr);
+      continue;
+    }
+    bitonic_sort_pairs<true>(skey, sidx, P);
     if (kk > 0) {
       const int PK = next_pow2(kk);
       for (int i = tid; i < PK; i += kThreads) ssel[i] = i < kk ? sidx[i] : 0x7fffffff;

@@ -40,6 +40,9 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kKeys = 64;     // pooled keys per shared-memory chunk
 constexpr int kGroups = kThreads / kKeys;  // row groups
+// Up to this many query blocks the routing splits by counted ranks (n comparisons per block),
+// above it by bitonic sorts.
+constexpr int kRankSplitMax = 512;
 
 __device__ __forceinline__ void store_elem(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void store_elem(float* p, float x) { *p = x; }
@@ -235,6 +238,17 @@ __global__ void __launch_bounds__(kThreads) route_kernel(Plan p, Work w) {
   if (!s_last) return;
   __threadfence();
 
+  const int n_flat = p.n_flat, n_exact = p.n_exact;
+  int32_t* route = w.route + (size_t)bh * n_q;
+  if (n_q <= kRankSplitMax) {
+    // rank of every (M_i, i) among all, then one scan: Taylor blocks (the n_flat lowest) and exact
+    // blocks, each in ascending block order
+    float* key = smem;
+    int32_t* scratch = reinterpret_cast<int32_t*>(key + n_q);
+    for (int i = tid; i < n_q; i += kThreads) key[i] = __ldcg(w.sharp + (size_t)bh * n_q + i);
+    rank_split<false>(key, n_q, n_flat, scratch, route + n_exact, route);
+    return;
+  }
   const int P = next_pow2(n_q);
   float* key = smem;                                       // [P]
   int32_t* idx = reinterpret_cast<int32_t*>(key + P);      // [P]
@@ -244,8 +258,6 @@ __global__ void __launch_bounds__(kThreads) route_kernel(Plan p, Work w) {
     idx[i] = i < n_q ? i : 0x7fffffff - (i - n_q);
   }
   bitonic_sort_pairs<false>(key, idx, P);
-  const int n_flat = p.n_flat, n_exact = p.n_exact;
-  int32_t* route = w.route + (size_t)bh * n_q;
   // exact part: ranks n_flat .. n_q-1, re-sorted by block index
   if (n_exact > 0) {
     const int PE = next_pow2(n_exact);
