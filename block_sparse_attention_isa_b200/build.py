@@ -49,7 +49,6 @@ REGISTER_SPLIT_KERNELS = {
     "attention_kernel": 168,
     "attention_mixed_kernel": 168,
     "attention_bwd_kernel": 168,
-    "attention_bwd_pair_kernel": 168,
 }
 
 

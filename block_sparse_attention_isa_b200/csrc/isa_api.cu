@@ -316,8 +316,38 @@ int host_pool(cudaMemPool_t* out) {
   return ISA_OK;
 }
 
-// The pass on host buffers: copies in, runs the pass (alpha_ns as for isa_forward_ns), copies
-// out and synchronises.
+// Streams of the host-buffer entry points, one set per device (created on first use): copies in,
+// the pass, copies out.
+struct HostStreams {
+  cudaStream_t in, comp, out;
+};
+int host_streams(HostStreams* out) {
+  static HostStreams streams[64] = {};
+  static bool made[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(ISA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!made[dev]) {
+    HostStreams hs;
+    if ((e = cudaStreamCreateWithFlags(&hs.in, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&hs.comp, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&hs.out, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "creating the library's streams");
+    streams[dev] = hs;
+    made[dev] = true;
+  }
+  *out = streams[dev];
+  return ISA_OK;
+}
+
+// The pass on host buffers (alpha_ns as for isa_forward_ns), synchronous. The (batch, head) slices
+// are independent, so the call runs as a pipeline over chunks of slices on three streams: the
+// inputs of chunk c + 1 are copied in while chunk c is computed and chunk c - 1 is copied out
+// (the two copy directions use separate copy engines), which hides the pass and the output copy
+// behind the input copy.
 int host_forward(const void* q, const void* k, const void* v, int B, int H, int L_src, int L_ctx, int D, int b,
                  float alpha_s, float alpha_f, float alpha_ns, isa_dtype dt, void* out, int32_t* dbg_sel,
                  int32_t* dbg_route) {
@@ -325,17 +355,36 @@ int host_forward(const void* q, const void* k, const void* v, int B, int H, int 
   int rc = make_plan(B, H, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &p, alpha_ns);
   if (rc != ISA_OK) return rc;
   if ((rc = check_io(q, k, v, out, p)) != ISA_OK) return rc;
+  // chunks of cs slices (about 8 chunks; the last may be smaller)
+  const int cs = (p.BH + 7) / 8;
+  const int nch = (p.BH + cs - 1) / cs;
+  Plan pc;  // plan of a full chunk (a chunk is the [1, cs, N, D] call of its slices)
+  if ((rc = make_plan(1, cs, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &pc, alpha_ns)) != ISA_OK) return rc;
   const size_t io = align256((size_t)p.BH * p.N * p.D * p.elem);
-  const size_t ws_bytes = workspace_layout(p, nullptr, nullptr);
+  const size_t ws_bytes = workspace_layout(pc, nullptr, nullptr);
   const size_t sel_b = align256(sizeof(int32_t) * (size_t)p.BH * (p.k > 0 ? p.k : 1));
   const size_t route_b = align256(sizeof(int32_t) * (size_t)p.BH * p.n_q);
   const size_t total = 4 * io + ws_bytes + sel_b + route_b;
-  cudaStream_t s = 0;
+  HostStreams hs;
+  if ((rc = host_streams(&hs)) != ISA_OK) return rc;
   cudaMemPool_t pool;
   if ((rc = host_pool(&pool)) != ISA_OK) return rc;
+  cudaEvent_t ev[2 * 8 + 2];
+  int n_ev = 0;
+  for (; n_ev < 2 * nch + 2; ++n_ev) {
+    const cudaError_t e = cudaEventCreateWithFlags(&ev[n_ev], cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      for (int i = 0; i < n_ev; ++i) cudaEventDestroy(ev[i]);
+      return cuda_fail(e, "creating events");
+    }
+  }
+  cudaEvent_t ev_alloc = ev[2 * nch], ev_end = ev[2 * nch + 1];
   char* dev_buf = nullptr;
-  cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&dev_buf), total, pool, s);
-  if (e != cudaSuccess) return cuda_fail(e, "allocating device buffers");
+  cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&dev_buf), total, pool, hs.comp);
+  if (e != cudaSuccess) {
+    for (int i = 0; i < n_ev; ++i) cudaEventDestroy(ev[i]);
+    return cuda_fail(e, "allocating device buffers");
+  }
   char* dq = dev_buf;
   char* dk = dq + io;
   char* dv = dk + io;
@@ -343,29 +392,67 @@ int host_forward(const void* q, const void* k, const void* v, int B, int H, int 
   char* dws = dout + io;
   int32_t* dsel = reinterpret_cast<int32_t*>(dws + ws_bytes);
   int32_t* droute = reinterpret_cast<int32_t*>(dws + ws_bytes + sel_b);
-  const size_t bytes = (size_t)p.BH * p.N * p.D * p.elem;
+  const size_t slice = (size_t)p.N * p.D * p.elem;
   rc = ISA_OK;
-  if ((e = cudaMemcpyAsync(dq, q, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(dk, k, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(dv, v, bytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
-    rc = cuda_fail(e, "copying inputs to the device");
-  if (rc == ISA_OK)
-    rc = run_forward(dq, dk, dv, p, dout, dbg_sel ? dsel : nullptr, dbg_route ? droute : nullptr, dws, ws_bytes, s);
-  if (rc == ISA_OK && (e = cudaMemcpyAsync(out, dout, bytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
-    rc = cuda_fail(e, "copying the output to the host");
-  if (rc == ISA_OK && dbg_sel && p.k > 0 &&
-      (e = cudaMemcpyAsync(dbg_sel, dsel, sizeof(int32_t) * (size_t)p.BH * p.k, cudaMemcpyDeviceToHost, s)) !=
-          cudaSuccess)
-    rc = cuda_fail(e, "copying dbg_sel to the host");
-  if (rc == ISA_OK && dbg_route &&
-      (e = cudaMemcpyAsync(dbg_route, droute, sizeof(int32_t) * (size_t)p.BH * p.n_q, cudaMemcpyDeviceToHost, s)) !=
-          cudaSuccess)
-    rc = cuda_fail(e, "copying dbg_route to the host");
-  const int st = read_status(dws, s);
+  if ((e = cudaEventRecord(ev_alloc, hs.comp)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(hs.in, ev_alloc, 0)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(hs.out, ev_alloc, 0)) != cudaSuccess)
+    rc = cuda_fail(e, "ordering the streams");
+  for (int c = 0; c < nch && rc == ISA_OK; ++c) {
+    const int s0 = c * cs, ns = (p.BH - s0) < cs ? (p.BH - s0) : cs;
+    const size_t off = (size_t)s0 * slice, nbytes = (size_t)ns * slice;
+    Plan pk = pc;
+    if (ns != cs && (rc = make_plan(1, ns, L_src, L_ctx, D, b, alpha_s, alpha_f, (int)dt, &pk, alpha_ns)) != ISA_OK)
+      break;
+    const char* hq = static_cast<const char*>(q) + off;
+    const char* hk = static_cast<const char*>(k) + off;
+    const char* hv = static_cast<const char*>(v) + off;
+    if ((e = cudaMemcpyAsync(dq + off, hq, nbytes, cudaMemcpyHostToDevice, hs.in)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dk + off, hk, nbytes, cudaMemcpyHostToDevice, hs.in)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dv + off, hv, nbytes, cudaMemcpyHostToDevice, hs.in)) != cudaSuccess ||
+        (e = cudaEventRecord(ev[2 * c], hs.in)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(hs.comp, ev[2 * c], 0)) != cudaSuccess) {
+      rc = cuda_fail(e, "copying inputs to the device");
+      break;
+    }
+    int32_t* csel = dsel + (size_t)s0 * p.k;
+    int32_t* croute = droute + (size_t)s0 * p.n_q;
+    rc = run_forward(dq + off, dk + off, dv + off, pk, dout + off, dbg_sel ? csel : nullptr,
+                     dbg_route ? croute : nullptr, dws, ws_bytes, hs.comp, /*keep_error=*/c > 0);
+    if (rc != ISA_OK) break;
+    if ((e = cudaEventRecord(ev[2 * c + 1], hs.comp)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(hs.out, ev[2 * c + 1], 0)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(static_cast<char*>(out) + off, dout + off, nbytes, cudaMemcpyDeviceToHost, hs.out)) !=
+            cudaSuccess) {
+      rc = cuda_fail(e, "copying the output to the host");
+      break;
+    }
+    if (dbg_sel && p.k > 0 &&
+        (e = cudaMemcpyAsync(dbg_sel + (size_t)s0 * p.k, csel, sizeof(int32_t) * (size_t)ns * p.k,
+                             cudaMemcpyDeviceToHost, hs.out)) != cudaSuccess) {
+      rc = cuda_fail(e, "copying dbg_sel to the host");
+      break;
+    }
+    if (dbg_route && (e = cudaMemcpyAsync(dbg_route + (size_t)s0 * p.n_q, croute,
+                                          sizeof(int32_t) * (size_t)ns * p.n_q, cudaMemcpyDeviceToHost, hs.out)) !=
+                         cudaSuccess) {
+      rc = cuda_fail(e, "copying dbg_route to the host");
+      break;
+    }
+  }
+  // whatever happened: the buffers are released only after every copy and kernel that uses them
+  if ((e = cudaEventRecord(ev_end, hs.out)) == cudaSuccess) e = cudaStreamWaitEvent(hs.comp, ev_end, 0);
+  if (e != cudaSuccess) {
+    cudaStreamSynchronize(hs.in);
+    cudaStreamSynchronize(hs.out);
+  }
+  cudaStreamSynchronize(hs.in);
+  const int st = read_status(dws, hs.comp);
   if (rc == ISA_OK) rc = st;
-  cudaFreeAsync(dev_buf, s);
-  e = cudaStreamSynchronize(s);
+  cudaFreeAsync(dev_buf, hs.comp);
+  e = cudaStreamSynchronize(hs.comp);
   if (rc == ISA_OK && e != cudaSuccess) rc = cuda_fail(e, "releasing device buffers");
+  for (int i = 0; i < n_ev; ++i) cudaEventDestroy(ev[i]);
   return rc;
 }
 

@@ -125,13 +125,6 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
                             const void* dout, void* dq, void* dk, void* dv, const Plan& pl, const Work& w,
                             void* bwd_ws, cudaStream_t s);
 
-// The backward kernels on CTA pairs (cta_group::2): whether their compiled register count is the
-// one their split needs, and the three launches after the delta pass.
-bool backward_pair_regs_ok();
-cudaError_t launch_backward_pair(const void* q, const void* k, const void* v, const void* dout, const Plan& pl,
-                                 const Work& w, const float* lse, const float* delta, void* dq, void* dk, void* dv,
-                                 float* dkc, float* dvc, cudaStream_t s);
-
 // One thread waits on an mbarrier that nothing arrives on; the bounded wait gives
 // up after `timeout_ms` and sets kErrSelftest in err[0].
 cudaError_t launch_wait_selftest(uint32_t* err, int timeout_ms, cudaStream_t s);

@@ -682,12 +682,6 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
                                                           static_cast<const __nv_bfloat16*>(out), delta, rows);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // the CTA-pair kernels (each CTA holds half of every column tile: half the L2 stream per row,
-  // and score MMAs not bound by shared-memory reads); the single-CTA ones below only when the
-  // pair kernels were compiled to another register count than their split needs
-  if (backward_pair_regs_ok())
-    return launch_backward_pair(q, k, v, dout, pl, w, lse, delta, dq, dk, dv, pl.n_flat > 0 ? dkc : nullptr,
-                                pl.n_flat > 0 ? dvc : nullptr, s);
   BwdParams p{};
   p.route = w.route;
   p.sel = w.sel;

@@ -110,6 +110,31 @@ def test_host_buffer_entry_matches_device_entry():
     np.testing.assert_array_equal(sel[0, 0].numpy(), ref["sel"])
 
 
+@pytest.mark.parametrize("pinned,a_ns", [(True, 0.0), (False, 0.0), (True, 0.25)])
+def test_host_buffer_pipeline_over_chunks(pinned, a_ns):
+    """The host-buffer entry point runs the (batch, head) slices in chunks on three streams (copy in,
+    pass, copy out). B = 2, H = 9: 18 slices in 6 chunks of 3; the result, the kept blocks and the
+    routing equal the device entry point's bit for bit, with pinned and pageable host buffers."""
+    import torch
+    import block_sparse_attention_isa_b200 as isa
+    from parity_util import to_device
+    w = _case("b128_b2_h9", 2, 9, 128, 512, 512, 128, 0.5, 0.5)
+    q, k, v = isa_synth.make_inputs(w, 0)
+    tq, tk, tv = (to_device(x, w) for x in (q, k, v))
+    dev = isa.forward(tq, tk, tv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, debug=True, alpha_ns=a_ns)
+    isa.device_status()
+    hq, hk, hv = (x.cpu() for x in (tq, tk, tv))
+    if pinned:
+        hq, hk, hv = (x.pin_memory() for x in (hq, hk, hv))
+    n_q, kk, _ = isa.plan(w.B, w.H, w.L_src, w.L_ctx, w.D, w.b, w.alpha_s, w.alpha_f)
+    sel = torch.full((w.B, w.H, kk), -1, dtype=torch.int32)
+    route = torch.full((w.B, w.H, n_q), -1, dtype=torch.int32)
+    host_out = isa.forward_host(hq, hk, hv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, dbg_sel=sel,
+                                dbg_route=route, alpha_ns=a_ns)
+    assert torch.equal(host_out, dev[0].cpu())
+    assert torch.equal(sel, dev[1].cpu()) and torch.equal(route, dev[2].cpu())
+
+
 def test_wait_timeout_is_reported_and_context_survives():
     import torch
     import block_sparse_attention_isa_b200 as isa
