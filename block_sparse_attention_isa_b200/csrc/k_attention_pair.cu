@@ -12,14 +12,13 @@
 // pooled rows. Each output row is written at its original token position.
 //
 // Why pairs. With one CTA per SM, every 256 query rows re-read their head's whole
-// K_new / V_new from L2 (22.5 GB per call at the 32K-token workload) and the
-// Q K^T MMAs read 8 KB of shared memory per 64 cycles, the tensor core's whole
-// shared-memory rate, so the K/V stream and the MMAs slow each other down. A
+// K_new / V_new from L2 (22.5 GB per call at the 32K-token workload). A
 // tcgen05.mma with cta_group::2 computes M = 256 rows on two SMs: each CTA holds
-// its own 128 query rows of A and HALF of B. Here each CTA loads 32 of the 64
+// its own 128 query rows of A and HALF of B. Here each CTA loads 64 of the 128
 // keys of every K tile and 64 of the 128 columns of every V tile, so per query
 // row the pair moves half the K/V bytes from L2 and reads half the B operand
-// bytes from shared memory.
+// bytes from shared memory (the Q K^T MMA, M = 256 and N = 128, then reads 6 KB
+// of shared memory per 64 cycles on each SM, under the 128 B/clk it can take).
 //
 // Structure (each CTA of the pair: 12 warps, one CTA per SM):
 //  * warp 0 issues the TMA loads of this CTA's halves; the loads of both CTAs
@@ -32,12 +31,18 @@
 //    peer (a slot with no tile for the peer gives it a copy of the leader's tile,
 //    computed and not stored). One thread per query row; every softmax thread of
 //    both CTAs arrives on the leader's "P written" barrier;
-//  * K/V tiles of 64 keys in 8-stage rings; TMEM of each CTA: slot t owns two
-//    64-column S buffers at [128 t, 128 t + 128) and O_t at [256 + 128 t, ...);
-//    S of K/V tile n goes to buffer n % 2, P_n is written over it as bf16 pairs
-//    and read by the P V MMA straight from TMEM;
-//  * MMA order per K/V tile j: P0 V_j, S0 of tile j + 2, P1 V_j, S1 of tile j + 2,
-//    so the softmax of tile j + 1 never waits for the P V of tile j;
+//  * K/V tiles of 128 keys in 4-stage rings; TMEM of each CTA: slot t owns one
+//    128-column S buffer at [128 t, 128 t + 128) and O_t at [256 + 128 t, ...);
+//    P_j is written over S_j as bf16 pairs (its first 64 columns) and read by the
+//    P V MMA straight from TMEM;
+//  * per slot, the MMA issuer sends P V_j and then S of tile j + 1 into the same
+//    buffer (one thread's MMAs run in issue order, so S_{j+1} is written only
+//    after P V_j has read P_j); the order per K/V tile is P0 V_j, S0 of j + 1,
+//    P1 V_j, S1 of j + 1, so while slot 0's softmax works on tile j + 1 the
+//    tensor core runs slot 1's P V and S, and the two softmax warpgroups stay
+//    staggered instead of sharing the ex2 units at the same time;
+//  * the softmax writes P in two halves of 64 keys and signals each, so the P V
+//    MMAs of the first half run while the second half is exponentiated;
 //  * lazy rescaling (the running max moves only when it grows by more than 2^8),
 //    exact items first and Taylor items after in the static schedule;
 //  * every wait is bounded; on a timeout the CTA flags an error in the device
@@ -69,16 +74,20 @@ constexpr int kHighRegs = 208;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
 constexpr int kD = 128;
 constexpr int kBM = 128;            // query rows per tile (per CTA)
-constexpr int kBN = 64;             // keys per K/V tile (per pair)
+constexpr int kBN = 128;            // keys per K/V tile (per pair)
 constexpr int kCols = kBN;          // scores per softmax thread and K/V tile
-constexpr int kStages = 8;   // K/V ring: stage i holds this CTA's halves of the K and V tile i
+#ifndef ISA_PAIR_STAGES
+#define ISA_PAIR_STAGES 4
+#endif
+constexpr int kStages = ISA_PAIR_STAGES;  // K/V ring: stage i holds this CTA's halves of the K and V tile i
 constexpr int kRB = kD * 2;         // bytes per row
 constexpr int kQCh = kBM * 128;     // bytes between the two 128-byte chunks of a Q tile
 constexpr int kQTile = kBM * kRB;   // 32 KB
 constexpr int kKRows = kBN / 2;     // keys of each K tile held by one CTA
 constexpr int kKCh = kKRows * 128;  // bytes between the chunks of a K half-tile
-constexpr int kKHalf = kKRows * kRB;  // 8 KB
-constexpr int kVHalf = kBN * 128;     // 8 KB: 64 keys x this CTA's 64 columns
+constexpr int kKHalf = kKRows * kRB;  // 16 KB
+constexpr int kVRows = 64;            // keys per V copy (a copy never straddles the seam of K_new)
+constexpr int kVHalf = kBN * 128;     // 16 KB: 128 keys x this CTA's 64 columns
 constexpr uint32_t kIdescQK = umma_idesc(1u, 256, kBN, 0, 0);
 constexpr uint32_t kIdescPV = umma_idesc(1u, 256, kD, 0, 1);
 constexpr float kRescaleThreshold = 8.0f;
@@ -121,11 +130,11 @@ struct Bars {
   uint64_t q_full[2];    // leader: Q of slot t in both CTAs
   uint64_t q_empty[2];   // slot t's S MMAs of the item are complete
   uint64_t kv_full[kStages];   // leader: both CTAs' K and V halves of the stage
-  uint64_t kv_empty[kStages];  // both MMA issuers are done with the stage (2 arrivals)
-  uint64_t s_full[2][2];  // [slot][S buffer]
-  uint64_t p_full[2][2];  // leader: [slot][S buffer], one arrival per softmax thread of both CTAs
-  uint64_t o_done[2][2];  // [slot][S buffer]: the P V MMAs of the K/V tiles in this buffer are complete
-  uint64_t drain[2];      // leader: every MMA of issuer t is complete
+  uint64_t kv_empty[kStages];  // the MMAs reading the stage are complete
+  uint64_t s_full[2];     // [slot]: S of the slot's next K/V tile (and every earlier MMA of it) complete
+  uint64_t p_full[2][2];  // leader: [slot][half], one arrival per softmax thread of both CTAs
+  uint64_t o_done[2];     // [slot]: the P V MMAs of the slot's item are complete
+  uint64_t drain;         // leader: every MMA is complete
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -162,7 +171,7 @@ __device__ __forceinline__ int qblock_len(const PairParams& p, int i) {
 __device__ __forceinline__ bool short_ctx_kept(const PairParams& p, const int32_t* sel, int bh) {
   return p.len_ctx_last < p.b && p.k > 0 && __ldg(sel + (size_t)bh * p.k + p.k - 1) == p.n_q - p.n_src - 1;
 }
-// -inf for the key rows [lo, hi) of the 64-key tile starting at row `base` (uniform per tile).
+// -inf for the key rows [lo, hi) of the K/V tile starting at row `base` (uniform per tile).
 __device__ __forceinline__ void mask_key_rows(uint32_t (&r)[kCols], int base, int lo, int hi) {
   if (hi <= base || lo >= base + kBN) return;
 #pragma unroll
@@ -263,17 +272,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->q_full[t], 1);
       mbar_init(&bars->q_empty[t], 1);
-      mbar_init(&bars->drain[t], 1);
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&bars->s_full[t][b], 1);
-        mbar_init(&bars->p_full[t][b], 256);
-        mbar_init(&bars->o_done[t][b], 1);
-      }
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->o_done[t], 1);
+      for (int h = 0; h < 2; ++h) mbar_init(&bars->p_full[t][h], 256);
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 2);
+      mbar_init(&bars->kv_empty[s], 1);
     }
+    mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -343,8 +350,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           if (rank == 0) mbar_arrive_expect_tx(&bars->kv_full[st], 2 * (kKHalf + kVHalf));
           const uint32_t bar = kv_full_l + 8u * st;
-          // K: this CTA's 32 keys of the tile (a 64-key tile never straddles the seam of K_new's
-          // source part, which ends at n_src * b)
+          // K: this CTA's 64 keys of the tile (64 keys never straddle the seam of K_new's source
+          // part, which ends at n_src * b, a multiple of 64)
           {
             const int rk = r0 + (int)rank * kKRows;
             const CUtensorMap* map;
@@ -357,16 +364,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 2; ++c) tma_load_pair(sK + st * kKHalf + c * kKCh, map, bar, c * 64, y, it.bh);
           }
-          // V: all 64 keys, this CTA's 64 columns
-          {
+          // V: all 128 keys in two copies of 64, this CTA's 64 columns
+#pragma unroll
+          for (int h = 0; h < kBN / kVRows; ++h) {
+            const int rv = r0 + h * kVRows;
             const CUtensorMap* map;
             int y;
             if (it.kind == 0) {
-              if (r0 < p.L_srcp) { map = &tm_v; y = r0; } else { map = &tm_vsel; y = r0 - p.L_srcp; }
+              if (rv < p.L_srcp) { map = &tm_v; y = rv; } else { map = &tm_vsel; y = rv - p.L_srcp; }
             } else {
-              map = &tm_vcn; y = r0;
+              map = &tm_vcn; y = rv;
             }
-            tma_load_pair(sV + st * kVHalf, map, bar, (int)rank * 64, y, it.bh);
+            tma_load_pair(sV + st * kVHalf + h * kVRows * 128, map, bar, (int)rank * 64, y, it.bh);
           }
         }
       }
@@ -379,47 +388,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1 || warp == 2) {
-    // ------------------------------------------------------------ MMA issuers (leader CTA only)
-    // Warp 1 issues the MMAs of slot 0 and warp 2 those of slot 1. The two streams are
-    // independent, so while one thread waits for a barrier the other keeps the tensor
-    // core busy (the issuing thread stalls on its barrier reads, and the MMA pipe holds
-    // little queued work). Both release each K/V stage (2 arrivals), so a thread whose
-    // slot is empty in an item still walks the item's stages, waiting for each to fill
-    // before releasing it: it can never release a stage ahead of the other thread.
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader CTA only)
+    // One thread issues the MMAs of both slots in a fixed order per K/V tile j:
+    // P0 V_j, S0 of tile j + 1, P1 V_j, S1 of tile j + 1. Slot 1's S completes one slot's
+    // worth of tensor work after slot 0's, so the two softmax warpgroups stay staggered:
+    // each exponentiates mostly while the tensor core runs the other slot's MMAs, rather
+    // than both at once on the shared ex2 units.
     if (rank == 0 && lane == 0) {
-      const int t = warp - 1;
       const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
-      uint32_t kv_base = 0, q_cnt = 0, s_seq = 0, p_seq = 0;
+      uint32_t kv_base = 0, q_cnt[2] = {0, 0}, p_seq[2] = {0, 0};
       bool ok = true;
       constexpr uint32_t HI = desc_hi_sw128(1024);
-      const uint32_t q_lo = desc_lo(smem_addr(sQ + t * kQTile), 16);
       const uint32_t k_lo = desc_lo(smem_addr(sK), 16);
       const uint32_t v_lo = desc_lo(smem_addr(sV), (uint32_t)kVHalf);
-      const uint32_t t_s = tmem + 128 * t, t_o = tmem + 256 + 128 * t;
-      // S = Q_t K^T for the K tile in stage st (rows of both CTAs, keys of both halves), into S buffer s_seq & 1
-      auto issue_s = [&](uint32_t st) {
-        const uint32_t d = t_s + (s_seq & 1) * kBN;
+      // S_t = Q_t K^T for the K tile in stage st (rows of both CTAs, keys of both halves)
+      auto issue_s = [&](int t, uint32_t st) {
+        const uint32_t q_lo = desc_lo(smem_addr(sQ + t * kQTile), 16);
         const uint32_t kb = k_lo + ((st * kKHalf) >> 4);
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           const uint32_t qo = (uint32_t)(((s / 4) * kQCh + (s % 4) * 32) >> 4);
           const uint32_t ko = (uint32_t)(((s / 4) * kKCh + (s % 4) * 32) >> 4);
-          mma_ss_pair(d, q_lo + qo, kb + ko, HI, kIdescQK, s > 0 ? 1u : 0u);
+          mma_ss_pair(tmem + 128 * t, q_lo + qo, kb + ko, HI, kIdescQK, s > 0 ? 1u : 0u);
         }
-        commit_pair(&bars->s_full[t][s_seq & 1]);
-        ++s_seq;
+        commit_pair(&bars->s_full[t]);
       };
-      // O_t (+)= P V for the V tile in stage st, P (of each CTA, from its own TMEM) in S buffer p_seq & 1
-      auto issue_pv = [&](uint32_t st, uint32_t acc) {
-        const uint32_t pa = t_s + (p_seq & 1) * kBN;
+      // O_t (+)= P V over keys [64 h, 64 h + 64) of the V tile in stage st, P (of each CTA, from its
+      // own TMEM) in slot t's S buffer columns [32 h, 32 h + 32)
+      auto issue_pv = [&](int t, uint32_t st, uint32_t acc, int h) {
         const uint32_t vb = v_lo + ((st * kVHalf) >> 4);
 #pragma unroll
-        for (int s = 0; s < kBN / 16; ++s)
-          mma_ts_pair(t_o, pa + s * 8, vb + (uint32_t)((s * 16 * 128) >> 4), HI, kIdescPV,
-                      (acc | (uint32_t)s) != 0 ? 1u : 0u);
-        commit_pair(&bars->o_done[t][p_seq & 1]);
-        ++p_seq;
+        for (int s = 4 * h; s < 4 * h + 4; ++s)
+          mma_ts_pair(tmem + 256 + 128 * t, tmem + 128 * t + s * 8, vb + (uint32_t)((s * 16 * 128) >> 4), HI,
+                      kIdescPV, (acc | (uint32_t)s) != 0 ? 1u : 0u);
       };
       auto wait = [&](uint64_t* bar, uint32_t par) -> bool {
         if (!mbar_wait_or_abort(bar, par, &bars->abort_flag)) {
@@ -432,46 +434,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       };
       for (int k = 0, g = schedule(p, pair, npairs, 0); g >= 0 && ok; g = schedule(p, pair, npairs, ++k)) {
         const Item it = decode_item(p, g);
-        const bool active = t < it.nslots;
-        if (active) {
-          if (!wait(&bars->q_full[t], q_cnt & 1)) break;
-          ++q_cnt;
-          // S of the first two K/V tiles (both S buffers)
-          const int pre = it.nkv < 2 ? it.nkv : 2;
-          for (int jj = 0; jj < pre; ++jj) {
-            const uint32_t idx = kv_base + jj, st = idx % kStages;
-            if (!wait(&bars->kv_full[st], (idx / kStages) & 1)) break;
-            issue_s(st);
-            if (jj == it.nkv - 1) commit_pair(&bars->q_empty[t]);
+        const int ns = it.nslots;
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (t < ns && ok && wait(&bars->q_full[t], q_cnt[t] & 1)) ++q_cnt[t];
+        if (!ok) break;
+        // S of the first K/V tile for every slot
+        {
+          const uint32_t st0 = kv_base % kStages;
+          if (!wait(&bars->kv_full[st0], (kv_base / kStages) & 1)) break;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (t >= ns) break;
+            issue_s(t, st0);
+            if (it.nkv == 1) commit_pair(&bars->q_empty[t]);
+          }
+        }
+        for (int j = 0; j < it.nkv && ok; ++j) {
+          const uint32_t idx = kv_base + j, st = idx % kStages;
+          const bool more = j + 1 < it.nkv;
+          const uint32_t idx1 = idx + 1, st1 = idx1 % kStages;
+          // the K/V stage of tile j + 1 first (normally long full)
+          if (more && !wait(&bars->kv_full[st1], (idx1 / kStages) & 1)) break;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (t >= ns) break;
+            if (!wait(&bars->p_full[t][0], p_seq[t] & 1)) break;
+            issue_pv(t, st, j > 0 ? 1u : 0u, 0);
+            if (!wait(&bars->p_full[t][1], p_seq[t] & 1)) break;
+            issue_pv(t, st, 1u, 1);
+            ++p_seq[t];
+            if (more) {
+              issue_s(t, st1);
+              if (j + 2 == it.nkv) commit_pair(&bars->q_empty[t]);
+            } else {
+              commit_pair(&bars->o_done[t]);
+            }
           }
           if (!ok) break;
-        }
-        // per K/V tile j: P V_j as soon as P is written, then S of tile j + 2 into the buffer
-        // that P V_j reads (one thread's MMAs run in issue order); then release stage j
-        for (int j = 0; j < it.nkv; ++j) {
-          const uint32_t idx = kv_base + j, st = idx % kStages;
-          if (active) {
-            // the K/V stage of tile j + 2 first (normally long full), so that PV_j and S_{j+2}
-            // go out back to back as soon as P_j is written
-            const bool more = j + 2 < it.nkv;
-            const uint32_t idx2 = idx + 2, st2 = idx2 % kStages;
-            if (more && !wait(&bars->kv_full[st2], (idx2 / kStages) & 1)) break;
-            if (!wait(&bars->p_full[t][p_seq & 1], (p_seq >> 1) & 1)) break;
-            issue_pv(st, j > 0 ? 1u : 0u);
-            if (more) {
-              issue_s(st2);
-              if (j + 3 == it.nkv) commit_pair(&bars->q_empty[t]);
-            }
-          } else {
-            if (!wait(&bars->kv_full[st], (idx / kStages) & 1)) break;
-          }
           commit_pair(&bars->kv_empty[st]);
         }
         kv_base += it.nkv;
       }
-      // every MMA this thread issued completes before either CTA can release TMEM or leave
-      commit_pair(&bars->drain[t]);
-      mbar_wait(&bars->drain[t], 0);
+      // every MMA completes before either CTA can release TMEM or leave
+      commit_pair(&bars->drain);
+      mbar_wait(&bars->drain, 0);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -485,11 +492,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t t_s = tmem + lane_off + t * 128;
     const uint32_t t_o = tmem + lane_off + 256 + t * 128;
     const uint32_t p_full_l = map_to(&bars->p_full[t][0], 0);  // the leader's P barriers of this slot
-    uint32_t seq = 0;
-    // wait until the P V MMA of sequence number n (and every earlier one) is complete; when this
-    // is called the one of n - 2 is known to be complete, so the buffer's barrier is at most one
-    // phase short of the one awaited
-    auto pv_done = [&](uint32_t n) { return warp_wait(bars, &bars->o_done[t][n & 1], (n >> 1) & 1, p.err); };
+    uint32_t seq = 0, items = 0;
     bool ok = true;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     for (int k = 0, g = schedule(p, pair, npairs, 0); g >= 0 && ok; g = schedule(p, pair, npairs, ++k)) {
@@ -498,11 +501,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool cs = kRagged ? short_ctx_kept(p, x.sel, it.bh) : false;
       float m = -FLT_MAX, l = 0.f;
       for (int j = 0; j < it.nkv; ++j, ++seq) {
-        const uint32_t buf = t_s + (seq & 1) * kBN;
-        if (!warp_wait(bars, &bars->s_full[t][seq & 1], (seq >> 1) & 1, p.err)) { ok = false; break; }
+        // S_j complete implies P V_{j-1} complete (the issuer sent it first), so O may be rescaled
+        if (!warp_wait(bars, &bars->s_full[t], seq & 1, p.err)) { ok = false; break; }
         uint32_t r[kCols];
-        tmem_ld32(buf, r);
-        tmem_ld32(buf + 32, r + 32);
+#pragma unroll
+        for (int c = 0; c < kCols / 32; ++c) tmem_ld32(t_s + 32 * c, r + 32 * c);
         tmem_ld_wait<kCols>(r);
         if (j == it.nkv - 1 && it.last_valid < kBN) {  // ragged last K/V tile (uniform branch)
 #pragma unroll
@@ -521,24 +524,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (cs) add_col_bias(r, j * kBN, p.n_new - 1, p.ctx_last_bias);
           }
         }
-        // row max: 8 independent chains of 3-input max over the 64 scores
+        // row max: 8 independent chains of 3-input max over the 128 scores
         float mc[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           mc[c] = fmax3(__uint_as_float(r[c]), __uint_as_float(r[8 + c]), __uint_as_float(r[16 + c]));
 #pragma unroll
-        for (int c = 0; c < 8; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[24 + c]), __uint_as_float(r[32 + c]));
+        for (int q = 24; q + 8 < kCols; q += 16)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[40 + c]), __uint_as_float(r[48 + c]));
+          for (int c = 0; c < 8; ++c) mc[c] = fmax3(mc[c], __uint_as_float(r[q + c]), __uint_as_float(r[q + 8 + c]));
 #pragma unroll
-        for (int c = 0; c < 8; ++c) mc[c] = fmaxf(mc[c], __uint_as_float(r[56 + c]));
+        for (int c = 0; c < 8; ++c) mc[c] = fmaxf(mc[c], __uint_as_float(r[kCols - 8 + c]));
         const float raw_max = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
         const float mx = raw_max * p.scale_log2;
         const bool need = (j > 0) && (mx > m + kRescaleThreshold);
         const float alpha = need ? ex2_approx(m - mx) : 1.0f;
         if (j == 0 || need) m = mx;
         if (__any_sync(0xffffffffu, need)) {
-          if (!pv_done(seq - 1)) { ok = false; break; }
 #pragma unroll 1
           for (int c = 0; c < kD / 32; ++c) {
             uint32_t o[32];
@@ -559,29 +561,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const float em = ex2_approx(fmaf(raw_max, p.scale_log2, -m));  // the largest p, as computed below
           corr = __bfloat162float(__float2bfloat16_rn(em)) - em;
         }
-        // p = 2^(s * scale - m) in pairs, written over this tile's S buffer as bf16 pairs
+        // p = 2^(s * scale - m) in pairs, written over this tile's S buffer as bf16 pairs, 64 keys
+        // (32 columns) at a time, each half signalled to the MMA issuer as soon as it is in TMEM
         const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(-m, -m);
         uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int i = 0; i < kCols / 2; ++i) {
-          const uint64_t x =
-              ffma2(static_cast<uint64_t>(r[2 * i]) | (static_cast<uint64_t>(r[2 * i + 1]) << 32), sc2, nm2);
-          const uint64_t e = (i % kPolyDen < kPolyNum) ? exp2_poly2(x) : pack2(ex2_approx(lo2(x)), ex2_approx(hi2(x)));
-          acc[i & 3] = fadd2(acc[i & 3], e);
-          __nv_bfloat162 hv = __floats2bfloat162_rn(lo2(e), hi2(e));
-          r[i] = *reinterpret_cast<uint32_t*>(&hv);
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int i = 32 * h; i < 32 * h + 32; ++i) {
+            const uint64_t x =
+                ffma2(static_cast<uint64_t>(r[2 * i]) | (static_cast<uint64_t>(r[2 * i + 1]) << 32), sc2, nm2);
+            const uint64_t e =
+                (i % kPolyDen < kPolyNum) ? exp2_poly2(x) : pack2(ex2_approx(lo2(x)), ex2_approx(hi2(x)));
+            acc[i & 3] = fadd2(acc[i & 3], e);
+            __nv_bfloat162 hv = __floats2bfloat162_rn(lo2(e), hi2(e));
+            r[i] = *reinterpret_cast<uint32_t*>(&hv);
+          }
+          tmem_st32(t_s + 32 * h, r + 32 * h);
+          tmem_st_wait();
+          tc_fence_before();
+          arrive_cluster(p_full_l + 8u * h);
         }
-        tmem_st32(buf, r);
-        tmem_st_wait();
-        tc_fence_before();
-        arrive_cluster(p_full_l + 8u * (seq & 1));
         const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
         l = l * alpha + ((lo2(a2) + hi2(a2)) + corr);
       }
       if (!ok) break;
       // epilogue: O / l at the row's original token position
       const float inv_l = 1.0f / l;
-      if (!pv_done(seq - 1)) { ok = false; break; }
+      if (!warp_wait(bars, &bars->o_done[t], items & 1, p.err)) { ok = false; break; }
+      ++items;
       const int ut = 2 * t + (int)rank;
       const int u = ut * p.bpt + row / p.b;
       const int qb = it.blk((ut < it.ntiles && u < it.nblk) ? u : 0);
@@ -683,9 +691,9 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
   const bool ok = make_map(&tq, q, 2, kD, pl.N, pl.BH, 64) && make_map(&tk, k, 2, kD, pl.N, pl.BH, kKRows) &&
                   make_map(&tks, has_sel ? w.ksel : k, 2, kD, sel_rows, pl.BH, kKRows) &&
                   make_map(&tkc, w.kcn, 2, kD, pl.n_new, pl.BH, kKRows) &&
-                  make_map(&tv, v, 2, kD, pl.N, pl.BH, kBN) &&
-                  make_map(&tvs, has_sel ? w.vsel : v, 2, kD, sel_rows, pl.BH, kBN) &&
-                  make_map(&tvc, w.vcn, 2, kD, pl.n_new, pl.BH, kBN);
+                  make_map(&tv, v, 2, kD, pl.N, pl.BH, kVRows) &&
+                  make_map(&tvs, has_sel ? w.vsel : v, 2, kD, sel_rows, pl.BH, kVRows) &&
+                  make_map(&tvc, w.vcn, 2, kD, pl.n_new, pl.BH, kVRows);
   if (!ok) return cudaErrorInvalidValue;
 
   auto kern = pl.ragged ? (w.lse ? attention_pair_kernel<true, true> : attention_pair_kernel<true, false>)
