@@ -531,8 +531,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
+    // The whole warp runs the loop with warp-uniform values; one elected lane issues each
+    // tensor-core instruction.
+    {
+      const uint32_t tmem = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base), 0);
       uint32_t kv_it = 0, q_cnt0 = 0, q_cnt1 = 0, pv_cnt0 = 0, pv_cnt1 = 0;
       bool ok = true;
       // descriptor low words of the operand bases; every K-step adds a compile-time offset
@@ -548,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           constexpr uint32_t dummy = 0;
           (void)dummy;
           const uint32_t off = (uint32_t)(((s / 4) * C::CH_STRIDE + (s % 4) * 32) >> 4);
-          umma_ss_lo<C::kTf32>(d, qa + off, ka + off, HI, C::IDESC_QK, s > 0 ? 1u : 0u);
+          umma_ss_lo_warp<C::kTf32>(d, qa + off, ka + off, HI, C::IDESC_QK, s > 0 ? 1u : 0u);
         }
       };
       // P V over keys [64 half, 64 half + 64) of the tile
@@ -557,11 +559,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = half * C::KS_PV / 2; s < (half + 1) * C::KS_PV / 2; ++s) {
           const uint32_t off = C::kVT ? (uint32_t)(((s / 4) * C::VT_CH_STRIDE + (s % 4) * 32) >> 4)
                                       : (uint32_t)((s * C::PV_K * 128) >> 4);
-          umma_ts_lo<C::kTf32>(d, pa + s * 8, va + off, HI, C::IDESC_PV, (acc | (uint32_t)s) != 0 ? 1u : 0u);
+          umma_ts_lo_warp<C::kTf32>(d, pa + s * 8, va + off, HI, C::IDESC_PV, (acc | (uint32_t)s) != 0 ? 1u : 0u);
         }
       };
       auto wait_or_abort = [&](uint64_t* bar, uint32_t par) -> bool {
-        if (!mbar_wait_or_abort(bar, par, &bars->abort_flag)) { raise_abort(bars, p.err, kErrMma); ok = false; return false; }
+        const bool got = mbar_wait_or_abort(bar, par, &bars->abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) raise_abort(bars, p.err, kErrMma);
+          ok = false;
+          return false;
+        }
         tc_fence_after();
         return true;
       };
@@ -583,13 +590,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!wait_or_abort(&bars->k_full[st], (kv_it / C::STAGES) & 1)) break;
           const uint32_t ka = st ? k_lo1 : k_lo0;
           issue_s(t_s0, q_lo0, ka);
-          umma_commit(&bars->s_full[0]);
+          umma_commit_warp(&bars->s_full[0]);
           if (two) {
             issue_s(t_s1, q_lo1, ka);
-            umma_commit(&bars->s_full[1]);
+            umma_commit_warp(&bars->s_full[1]);
           }
-          umma_commit(&bars->k_empty[st]);
-          if (it.nkv == 1) umma_commit(&bars->q_empty);
+          umma_commit_warp(&bars->k_empty[st]);
+          if (it.nkv == 1) umma_commit_warp(&bars->q_empty);
         }
         for (int j = 0; j < it.nkv; ++j, ++kv_it) {
           const uint32_t st = kv_it % C::STAGES;
@@ -602,17 +609,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             // were consumed by its last P V, issued earlier).
             if (more) {
               if (!wait_or_abort(&bars->k_full[st1], ((kv_it + 1) / C::STAGES) & 1)) break;
-              const uint32_t tiles = *reinterpret_cast<volatile uint32_t*>(&bars->stage_tiles[st1]);
+              const uint32_t tiles =
+                  __shfl_sync(0xffffffffu, *reinterpret_cast<volatile uint32_t*>(&bars->stage_tiles[st1]), 0);
               pn0 = (tiles & 1u) != 0u;
               pn1 = two && (tiles & 2u) != 0u;
               const uint32_t ka1 = st1 ? k_lo1 : k_lo0;
               if (!pc0 && pn0) {
                 issue_s(t_s0, q_lo0, ka1);
-                umma_commit(&bars->s_full[0]);
+                umma_commit_warp(&bars->s_full[0]);
               }
               if (!pc1 && pn1) {
                 issue_s(t_s1, q_lo1, ka1);
-                umma_commit(&bars->s_full[1]);
+                umma_commit_warp(&bars->s_full[1]);
               }
             }
           }
@@ -626,14 +634,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_pv(t_o0, t_s0, va, acc, 0);
             if (!wait_or_abort(&bars->p_half[0][1], pv_cnt0 & 1)) break;
             issue_pv(t_o0, t_s0, va, 1u, 1);
-            umma_commit(&bars->o_done[0]);
+            umma_commit_warp(&bars->o_done[0]);
             ++pv_cnt0;
           }
           if (more) {
             if (!NS && !wait_or_abort(&bars->k_full[st1], ((kv_it + 1) / C::STAGES) & 1)) break;
             if (!NS || (pc0 && pn0)) {
               issue_s(t_s0, q_lo0, ka1);
-              umma_commit(&bars->s_full[0]);
+              umma_commit_warp(&bars->s_full[0]);
             }
           }
           // tile 1
@@ -642,24 +650,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_pv(t_o1, t_s1, va, acc, 0);
             if (!wait_or_abort(&bars->p_half[1][1], pv_cnt1 & 1)) break;
             issue_pv(t_o1, t_s1, va, 1u, 1);
-            umma_commit(&bars->o_done[1]);
+            umma_commit_warp(&bars->o_done[1]);
             ++pv_cnt1;
           }
           if (NS ? (pc1 && pn1) : (two && more)) {
             issue_s(t_s1, q_lo1, ka1);
-            umma_commit(&bars->s_full[1]);
+            umma_commit_warp(&bars->s_full[1]);
           }
           if (more) {
-            umma_commit(&bars->k_empty[st1]);
-            if (j + 2 == it.nkv) umma_commit(&bars->q_empty);
+            umma_commit_warp(&bars->k_empty[st1]);
+            if (j + 2 == it.nkv) umma_commit_warp(&bars->q_empty);
           }
-          umma_commit(&bars->v_empty[st]);
+          umma_commit_warp(&bars->v_empty[st]);
           pc0 = pn0;
           pc1 = pn1;
         }
       }
       // every MMA issued by this thread completes before TMEM can be released
-      umma_commit(&bars->drain);
+      umma_commit_warp(&bars->drain);
       mbar_wait(&bars->drain, 0);
     }
     __syncwarp();

@@ -326,15 +326,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
+    // The whole warp runs the loop with warp-uniform values; one elected lane issues each
+    // tensor-core instruction.
+    {
+      const uint32_t tmem = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base), 0);
       constexpr uint32_t HI = desc_hi_sw128(1024);
       const uint32_t a1_lo = desc_lo(smem_addr(sA1), 16), a2_lo = desc_lo(smem_addr(sA2), 16);
       uint32_t n_items = 0, tile_it = 0, ct = 0;
       bool ok = true;
       auto wait = [&](uint64_t* bar, uint32_t par) -> bool {
-        if (!mbar_wait_or_abort(bar, par, &bars->abort_flag)) {
-          raise_abort(bars, p.err, kErrMma);
+        const bool got = mbar_wait_or_abort(bar, par, &bars->abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) raise_abort(bars, p.err, kErrMma);
           ok = false;
           return false;
         }
@@ -347,14 +350,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 8; ++s) {
           const uint32_t oa = (uint32_t)(((s / 4) * kACh + (s % 4) * 32) >> 4);
           const uint32_t ob = (uint32_t)(((s / 4) * kBCh + (s % 4) * 32) >> 4);
-          umma_ss_lo<false>(d, a_lo + oa, b_lo + ob, HI, kIdescS, s > 0 ? 1u : 0u);
+          umma_ss_lo_warp<false>(d, a_lo + oa, b_lo + ob, HI, kIdescS, s > 0 ? 1u : 0u);
         }
       };
       // D (128 x 128) (+)= X (TMEM, 128 x 64 bf16) * B (64 x 128, MN-major)
       auto issue_acc = [&](uint32_t d, uint32_t x_tmem, uint32_t b_lo, uint32_t acc) {
 #pragma unroll
         for (int s = 0; s < kBN / 16; ++s)
-          umma_ts_lo<false>(d, x_tmem + s * 8, b_lo + (uint32_t)((s * 16 * 128) >> 4), HI, kIdescAcc,
+          umma_ts_lo_warp<false>(d, x_tmem + s * 8, b_lo + (uint32_t)((s * 16 * 128) >> 4), HI, kIdescAcc,
                             (acc | (uint32_t)s) != 0 ? 1u : 0u);
       };
       const uint32_t t_s = tmem, t_t = tmem + 128, t_acc0 = tmem + 256, t_acc1 = tmem + 384;
@@ -376,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t bf = ct & 1;
             issue_score(t_s + bf * kBN, a1_lo, b1);
             issue_score(t_t + bf * kBN, a2_lo, b2);
-            umma_commit(&bars->s_full[bf]);
-            if (jj == nc - 1) umma_commit(&bars->a_empty);
+            umma_commit_warp(&bars->s_full[bf]);
+            if (jj == nc - 1) umma_commit_warp(&bars->a_empty);
           }
           if (jj > 0) {
             // the accumulating MMAs of tile jj - 1 once its P and dS are in TMEM
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               issue_acc(t_acc0, t_t + bf * kBN, b1, acc);  // dQ += dS K
             }
-            umma_commit(&bars->kv_empty[prev_st]);
+            umma_commit_warp(&bars->kv_empty[prev_st]);
           }
           if (jj < nc) {
             prev_st = tile_it % kStages;
@@ -403,10 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        umma_commit(&bars->acc_full);
+        umma_commit_warp(&bars->acc_full);
       }
       // every MMA issued by this thread completes before TMEM can be released
-      umma_commit(&bars->drain);
+      umma_commit_warp(&bars->drain);
       mbar_wait(&bars->drain, 0);
     }
     __syncwarp();

@@ -237,15 +237,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
+    // The whole warp runs the loop with warp-uniform values; one elected lane issues each
+    // tensor-core instruction.
+    {
+      const uint32_t tmem = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base), 0);
       constexpr uint32_t HI = desc_hi_sw128(1024);
       const uint32_t q_lo = desc_lo(smem_addr(sQ), 16);
-      uint32_t n_items = 0, kv_it = 0, s_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
+      uint32_t n_items = 0, kv_it = 0;
+      uint32_t pv_par = 0;  // bit w: parity of the number of P V groups issued for warpgroup w
       bool ok = true;
       auto wait = [&](uint64_t* bar, uint32_t par) -> bool {
-        if (!mbar_wait_or_abort(bar, par, &bars->abort_flag)) {
-          raise_abort(bars, p.err, kErrMma);
+        const bool got = mbar_wait_or_abort(bar, par, &bars->abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) raise_abort(bars, p.err, kErrMma);
           ok = false;
           return false;
         }
@@ -258,20 +262,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           const uint32_t off = (uint32_t)(((s / 4) * kCh + (s % 4) * 32) >> 4);
-          umma_ss_lo<false>(tmem + 128 * w, q_lo + off, k_lo + off, HI, kIdescQK, s > 0 ? 1u : 0u);
+          umma_ss_lo_warp<false>(tmem + 128 * w, q_lo + off, k_lo + off, HI, kIdescQK, s > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->s_full[w]);
-        ++s_cnt[w];
+        umma_commit_warp(&bars->s_full[w]);
       };
       // O_w (+)= P_w V for the V tile of stage st
       auto issue_pv = [&](int w, uint32_t st, uint32_t acc) {
         const uint32_t v_lo = desc_lo(smem_addr(sKV + st * 2 * kTile + kTile), (uint32_t)kCh);
 #pragma unroll
         for (int s = 0; s < kBN / 16; ++s)
-          umma_ts_lo<false>(tmem + 256 + 128 * w, tmem + 128 * w + s * 8, v_lo + (uint32_t)((s * 16 * 128) >> 4), HI,
+          umma_ts_lo_warp<false>(tmem + 256 + 128 * w, tmem + 128 * w + s * 8, v_lo + (uint32_t)((s * 16 * 128) >> 4), HI,
                             kIdescPV, (acc | (uint32_t)s) != 0 ? 1u : 0u);
-        umma_commit(&bars->o_done[w]);
-        ++pv_cnt[w];
+        umma_commit_warp(&bars->o_done[w]);
+        pv_par ^= 1u << w;
       };
       for (int g = blockIdx.x; g < total && ok; g += gridDim.x, ++n_items) {
         const Item it = decode_item(p, g);
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t idx = kv_it + j, st = idx % kStages;
           if (!wait(&bars->kv_full[st], (idx / kStages) & 1)) break;
           issue_s(j & 1, st);
-          if (j == it.nkv - 1) umma_commit(&bars->q_empty);
+          if (j == it.nkv - 1) umma_commit_warp(&bars->q_empty);
         }
         if (!ok) break;
         // the O accumulators of the previous item have been read by the merge
@@ -290,19 +293,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int w = j & 1;
           const uint32_t idx = kv_it + j, st = idx % kStages;
           // P V of tile j once its P is written, then S of tile j + 2 into the buffer it read
-          if (!wait(&bars->p_full[w], (pv_cnt[w]) & 1)) break;
+          if (!wait(&bars->p_full[w], (pv_par >> w) & 1u)) break;
           issue_pv(w, st, j >= 2 ? 1u : 0u);
-          umma_commit(&bars->kv_empty[st]);
+          umma_commit_warp(&bars->kv_empty[st]);
           if (j + 2 < it.nkv) {
             const uint32_t idx2 = idx + 2, st2 = idx2 % kStages;
             if (!wait(&bars->kv_full[st2], (idx2 / kStages) & 1)) break;
             issue_s(w, st2);
-            if (j + 3 == it.nkv) umma_commit(&bars->q_empty);
+            if (j + 3 == it.nkv) umma_commit_warp(&bars->q_empty);
           }
         }
         kv_it += it.nkv;
       }
-      umma_commit(&bars->drain);
+      umma_commit_warp(&bars->drain);
       mbar_wait(&bars->drain, 0);
     }
     __syncwarp();

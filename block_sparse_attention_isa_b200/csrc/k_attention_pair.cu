@@ -92,9 +92,10 @@ constexpr uint32_t kIdescQK = umma_idesc(1u, 256, kBN, 0, 0);
 constexpr uint32_t kIdescPV = umma_idesc(1u, 256, kD, 0, 1);
 constexpr float kRescaleThreshold = 8.0f;
 // Share of the exponentials computed by the FMA-pipe polynomial (exp2_poly.cuh) instead of
-// ex2: pair i of a row goes to the polynomial when (i % kPolyDen) < kPolyNum.
+// ex2: pair i of a row goes to the polynomial when (i % kPolyDen) < kPolyNum. One pair in eight
+// measured 1.5-2.5 % faster than none; two in eight slower again.
 #ifndef ISA_PAIR_POLY_NUM
-#define ISA_PAIR_POLY_NUM 0
+#define ISA_PAIR_POLY_NUM 1
 #endif
 #ifndef ISA_PAIR_POLY_DEN
 #define ISA_PAIR_POLY_DEN 8
@@ -390,13 +391,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader CTA only)
-    // One thread issues the MMAs of both slots in a fixed order per K/V tile j:
+    // The whole warp runs the issue loop with warp-uniform values and one elected lane issues
+    // each tensor-core instruction (issued from a single-lane branch, every MMA took about 60
+    // cycles of the issuing thread, as long as the MMA itself). The MMAs of both slots go out
+    // in a fixed order per K/V tile j:
     // P0 V_j, S0 of tile j + 1, P1 V_j, S1 of tile j + 1. Slot 1's S completes one slot's
     // worth of tensor work after slot 0's, so the two softmax warpgroups stay staggered:
     // each exponentiates mostly while the tensor core runs the other slot's MMAs, rather
     // than both at once on the shared ex2 units.
-    if (rank == 0 && lane == 0) {
-      const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base);
+    if (rank == 0) {
+      const uint32_t tmem = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile uint32_t*>(&bars->tmem_base), 0);
       uint32_t kv_base = 0, q_cnt[2] = {0, 0}, p_seq[2] = {0, 0};
       bool ok = true;
       constexpr uint32_t HI = desc_hi_sw128(1024);
@@ -410,9 +414,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 8; ++s) {
           const uint32_t qo = (uint32_t)(((s / 4) * kQCh + (s % 4) * 32) >> 4);
           const uint32_t ko = (uint32_t)(((s / 4) * kKCh + (s % 4) * 32) >> 4);
-          mma_ss_pair(tmem + 128 * t, q_lo + qo, kb + ko, HI, kIdescQK, s > 0 ? 1u : 0u);
+          mma_ss_pair_warp(tmem + 128 * t, q_lo + qo, kb + ko, HI, kIdescQK, s > 0 ? 1u : 0u);
         }
-        commit_pair(&bars->s_full[t]);
+        commit_pair_warp(&bars->s_full[t]);
       };
       // O_t (+)= P V over keys [64 h, 64 h + 64) of the V tile in stage st, P (of each CTA, from its
       // own TMEM) in slot t's S buffer columns [32 h, 32 h + 32)
@@ -420,12 +424,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t vb = v_lo + ((st * kVHalf) >> 4);
 #pragma unroll
         for (int s = 4 * h; s < 4 * h + 4; ++s)
-          mma_ts_pair(tmem + 256 + 128 * t, tmem + 128 * t + s * 8, vb + (uint32_t)((s * 16 * 128) >> 4), HI,
+          mma_ts_pair_warp(tmem + 256 + 128 * t, tmem + 128 * t + s * 8, vb + (uint32_t)((s * 16 * 128) >> 4), HI,
                       kIdescPV, (acc | (uint32_t)s) != 0 ? 1u : 0u);
       };
       auto wait = [&](uint64_t* bar, uint32_t par) -> bool {
-        if (!mbar_wait_or_abort(bar, par, &bars->abort_flag)) {
-          raise_abort(bars, p.err, kErrMma);
+        const bool got = mbar_wait_or_abort(bar, par, &bars->abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) raise_abort(bars, p.err, kErrMma);
           ok = false;
           return false;
         }
@@ -447,7 +452,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 2; ++t) {
             if (t >= ns) break;
             issue_s(t, st0);
-            if (it.nkv == 1) commit_pair(&bars->q_empty[t]);
+            if (it.nkv == 1) commit_pair_warp(&bars->q_empty[t]);
           }
         }
         for (int j = 0; j < it.nkv && ok; ++j) {
@@ -466,19 +471,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ++p_seq[t];
             if (more) {
               issue_s(t, st1);
-              if (j + 2 == it.nkv) commit_pair(&bars->q_empty[t]);
+              if (j + 2 == it.nkv) commit_pair_warp(&bars->q_empty[t]);
             } else {
-              commit_pair(&bars->o_done[t]);
+              commit_pair_warp(&bars->o_done[t]);
             }
           }
           if (!ok) break;
-          commit_pair(&bars->kv_empty[st]);
+          commit_pair_warp(&bars->kv_empty[st]);
         }
         kv_base += it.nkv;
       }
       // every MMA completes before either CTA can release TMEM or leave
-      commit_pair(&bars->drain);
+      commit_pair_warp(&bars->drain);
       mbar_wait(&bars->drain, 0);
+      __syncwarp();
     }
     __syncwarp();
   } else if (warp >= 4) {

@@ -67,4 +67,34 @@ __device__ __forceinline__ void mma_ts_pair(uint32_t d, uint32_t a_tmem, uint32_
       : "memory");
 }
 
+// The same three instructions for a converged warp: every lane runs them with the same
+// (warp-uniform) operands and elect.sync picks the one lane that issues (as the cta_group::1
+// forms in ptx.cuh, and for the same reason).
+__device__ __forceinline__ void commit_pair_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}\n" ::"r"(
+          smem_addr(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ss_pair_warp(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                                 uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .b64 da, db;\n\t.reg .pred p, e;\n\tmov.b64 da, {%1, %5};\n\tmov.b64 db, {%2, %5};\n\t"
+      "setp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %3, p;\n\t}\n" ::"r"(d),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(acc), "r"(hi)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_pair_warp(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                                 uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .b64 db;\n\t.reg .pred p, e;\n\tmov.b64 db, {%2, %5};\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], db, %3, p;\n\t}\n" ::"r"(d),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(acc), "r"(hi)
+      : "memory");
+}
+
 }  // namespace isa
