@@ -80,7 +80,11 @@ enum : uint32_t {
 };
 
 // Control words at the start of the workspace (cleared on every call).
-enum : int { kCtrlError = 0, kCtrlGridBarrier = 1 };
+enum : int {
+  kCtrlError = 0,
+  kCtrlGridBarrier = 1,
+  kCtrlMixedNext = 2,  // next work item of the mixed Taylor kernel (dynamic schedule)
+};
 
 // Floats of the pooling kernel's per-item partial sums for these sizes.
 size_t pool_partial_floats(const Plan& p);

@@ -48,6 +48,7 @@ constexpr int kCh = 128 * 128;        // bytes between the two 128-byte chunks o
 constexpr uint32_t kIdescQK = umma_idesc(1u, 128, kBN, 0, 0);
 constexpr uint32_t kIdescPV = umma_idesc(1u, 128, kD, 0, 1);
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kRing = 4;  // work items published ahead by the producer
 
 struct MixParams {
   const int32_t* route;    // [BH, n_q]: exact blocks, then Taylor blocks
@@ -55,6 +56,7 @@ struct MixParams {
   const uint32_t* nsmask;  // [BH, n_q, ns_words]: the same as a bitmask over K_new's blocks
   void* out;
   uint32_t* err;
+  uint32_t* next;          // per-call work counter (zeroed with the control words)
   int BH, N, n_q, n_src, n_exact, n_flat, n_new, k_ns, ns_words, npt;
   float scale_log2;
   float bias_log2;         // log2(b): a pooled row's weight b in the exponent
@@ -68,6 +70,9 @@ struct Bars {
   uint64_t st_full;        // warpgroup 1 has written m1, l1 of the item (128 arrivals)
   uint64_t st_read;        // warpgroup 0 has read them (128 arrivals)
   uint64_t drain;
+  uint64_t item_full[kRing];  // the producer has published the item in the slot
+  uint64_t item_free[kRing];  // the issuer (1) and the softmax threads (256) have read it
+  int item_ring[kRing];       // item index, or -1 past the last
   uint32_t tmem_base;
   int abort_flag;
   float m1[128], l1[128];  // warpgroup 1's softmax state per row, for the merge
@@ -150,6 +155,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->st_full, 128);
     mbar_init(&bars->st_read, 128);
     mbar_init(&bars->drain, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&bars->item_full[i], 1);
+      mbar_init(&bars->item_free[i], 257);
+    }
     bars->abort_flag = 0;
     mbar_fence_init();
   }
@@ -177,7 +186,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t n_items = 0, kv_it = 0;
       bool ok = true;
-      for (int g = blockIdx.x; g < total && ok; g += gridDim.x, ++n_items) {
+      // Items come from a per-call counter (a CTA that starts late, on an SM freed late by the
+      // kernel before, takes fewer), published to the other roles through the ring.
+      for (uint32_t n = 0; ok; ++n, ++n_items) {
+        const uint32_t slot = n % kRing;
+        if (n >= kRing && !mbar_wait(&bars->item_free[slot], ((n / kRing) - 1) & 1)) {
+          raise_abort(bars, p.err, kErrProducer);
+          ok = false;
+          break;
+        }
+        int g = (int)atomicAdd(p.next, 1u);
+        if (g >= total) g = -1;
+        *reinterpret_cast<volatile int*>(&bars->item_ring[slot]) = g;
+        mbar_arrive(&bars->item_full[slot]);
+        if (g < 0) break;
         const Item it = decode_item(p, g);
         if (n_items > 0 && !mbar_wait(&bars->q_empty, (n_items - 1) & 1)) {
           raise_abort(bars, p.err, kErrProducer);
@@ -276,7 +298,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit_warp(&bars->o_done[w]);
         pv_par ^= 1u << w;
       };
-      for (int g = blockIdx.x; g < total && ok; g += gridDim.x, ++n_items) {
+      for (uint32_t n = 0; ok; ++n, ++n_items) {
+        const uint32_t slot = n % kRing;
+        if (!wait(&bars->item_full[slot], (n / kRing) & 1)) break;
+        const int g = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&bars->item_ring[slot]), 0);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->item_free[slot]);
+        if (g < 0) break;
         const Item it = decode_item(p, g);
         if (!wait(&bars->q_full, n_items & 1)) break;
         // S of the first two key tiles (one per warpgroup)
@@ -323,7 +351,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     constexpr uint32_t kNegInf = 0xff800000u;
-    for (int g = blockIdx.x; g < total && ok; g += gridDim.x, ++n_items) {
+    for (uint32_t n = 0; ok; ++n, ++n_items) {
+      const uint32_t slot = n % kRing;
+      if (!warp_wait(bars, &bars->item_full[slot], (n / kRing) & 1, p.err)) { ok = false; break; }
+      const int g = *reinterpret_cast<volatile int*>(&bars->item_ring[slot]);
+      mbar_arrive(&bars->item_free[slot]);
+      if (g < 0) break;
       const Item it = decode_item(p, g);
       const uint32_t* own = p.nsmask + ((size_t)it.bh * p.n_q + it.blk) * p.ns_words;
       float m = -INFINITY, l = 0.f;
@@ -458,6 +491,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(*reinterpret_cast<volatile uint32_t*>(&bars->tmem_base), 512);
   }
+  // This grid may start before the attention kernel launched ahead of it has finished (it takes
+  // the SMs that kernel frees); it does not read that kernel's output, but it finishes only after
+  // it, so that stream order holds for the work after both.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace
@@ -474,6 +511,7 @@ cudaError_t launch_attention_mixed(const void* q, const void* k, const void* v, 
   p.nsmask = w.nsmask;
   p.out = out;
   p.err = w.ctrl;
+  p.next = w.ctrl + kCtrlMixedNext;
   p.BH = pl.BH;
   p.N = pl.N;
   p.n_q = pl.n_q;
@@ -507,8 +545,19 @@ cudaError_t launch_attention_mixed(const void* q, const void* k, const void* v, 
     return e;
   int grid = device_sm_count();
   if (grid > total) grid = total;
-  kern<<<grid, kThreads, kSmemAlloc, s>>>(tq, tk, tks, tv, tvs, tkc, tvc, p);
-  return cudaGetLastError();
+  // Programmatic dependent launch: the CTAs may start on the SMs the preceding attention kernel
+  // frees (that kernel allows it at its start) instead of after its last CTA.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tq, tk, tks, tv, tvs, tkc, tvc, p);
 }
 
 }  // namespace isa

@@ -305,6 +305,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_warp();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
 
+  // A kernel launched after this one with programmatic serialization (the mixed Taylor kernel)
+  // may take SMs as soon as CTAs of this grid exit.
+  asm volatile("griddepcontrol.launch_dependents;");
+
   if (warp < 4) regs_dealloc<kLowRegs>();
 
   if (warp == 0) {
