@@ -99,6 +99,22 @@ def test_small_full_parity_ns(w, a_ns):
     compare_out(out, ref["out"])
 
 
+def test_alpha_ns_repeat_runs_bit_identical():
+    """The mixed Taylor kernel takes its work items from a per-call counter, so which CTA computes an
+    item changes from run to run; every item is computed whole by one CTA, so the outputs may not."""
+    import torch
+    import block_sparse_attention_isa_b200 as isa
+    w = _case("b128_h8", 1, 8, 128, 4096, 4096, 128, 0.25, 0.6)
+    q, k, v = ns_inputs(w, 0.0625)
+    tq, tk, tv = (to_device(x, w) for x in (q, k, v))
+    runs = [isa.forward(tq, tk, tv, w.L_src, w.L_ctx, w.b, w.alpha_s, w.alpha_f, debug=True, alpha_ns=0.0625)
+            for _ in range(3)]
+    isa.device_status()
+    for other in runs[1:]:
+        for x, y in zip(runs[0], other):
+            assert torch.equal(x, y)
+
+
 def test_alpha_ns_zero_equals_plain_entry():
     """isa_forward_ns with alpha_ns = 0 runs exactly the plain pass (bit-identical outputs)."""
     import torch
