@@ -478,10 +478,14 @@ def run_ours(args, w):
                          "flops_share": {"exact": f["exact"] / (f["exact"] + f["taylor"]),
                                          "taylor": f["taylor"] / (f["exact"] + f["taylor"])},
                          "traffic": traffic},
+            # time x (median SM clock / max clock): what the stage would take at the max clock if it
+            # scaled with the clock alone, against the burst peak (the one measured near the max
+            # clock; the sustained peak was measured at the power-capped clock)
             "clock_normalised": None if clock_ratio is None else {
                 "sm_mhz_median": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                 "attention_ms_at_max_clock": stage_ms["attention"] * clock_ratio,
-                "frac_at_max_clock": attn_tflops / clock_ratio / peak},
+                "frac_at_max_clock": attn_tflops / clock_ratio / peaks["bf16_tflops"],
+                "peak_kind": "measured bf16 burst" if peaks_kind == "measured" else "fallback bf16 burst"},
             "pass_roofline": {"measured": pass_roofline(f, hb, ms, peak, peaks["hbm_gbs"]),
                               "nominal": pass_roofline(f, hb, ms, NOMINAL["bf16_tflops"], NOMINAL["hbm_gbs"])},
             "stages_ms": stage_ms,
