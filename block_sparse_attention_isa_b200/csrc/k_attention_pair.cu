@@ -24,8 +24,10 @@
 //  * warp 0 issues the TMA loads of this CTA's halves; the loads of both CTAs
 //    signal the leader CTA's "full" barriers, which the leader arms with the
 //    byte count of both halves;
-//  * warp 1 of the leader issues every MMA from one thread; completions are
-//    committed to the barriers of both CTAs at once (multicast commit);
+//  * warp 1 of the leader issues every MMA: the whole warp runs the loop with
+//    warp-uniform values and one elected lane issues each instruction (the MMAs
+//    go out in one order, from one lane at a time); completions are committed
+//    to the barriers of both CTAs at once (multicast commit);
 //  * warps 4-7 and 8-11 are two softmax warpgroups per CTA, one per query-tile
 //    slot: slot t of a work item is tile 2t in the leader and tile 2t + 1 in the
 //    peer (a slot with no tile for the peer gives it a copy of the leader's tile,
@@ -44,7 +46,8 @@
 //  * the softmax writes P in two halves of 64 keys and signals each, so the P V
 //    MMAs of the first half run while the second half is exponentiated;
 //  * lazy rescaling (the running max moves only when it grows by more than 2^8),
-//    exact items first and Taylor items after in the static schedule;
+//    exact items first and Taylor items after in the static schedule; one pair
+//    of exponentials in eight on the FMA-pipe polynomial (exp2_poly.cuh);
 //  * every wait is bounded; on a timeout the CTA flags an error in the device
 //    error word and in the abort flags of both CTAs, lets its copies land,
 //    meets its peer at a cluster barrier and frees TMEM.
