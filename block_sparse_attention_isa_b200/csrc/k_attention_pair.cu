@@ -569,11 +569,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // dominant keys have p in (1, 2^8] (only in tiles whose maximum exceeds m), which bf16
         // rounds by up to 2^-9: left in the sum, that mismatch between numerator and denominator
         // would scale the whole output row by it. (A key that set m has p = 1 exactly.)
-        float corr = 0.f;
-        if (mx > m) {
-          const float em = ex2_approx(fmaf(raw_max, p.scale_log2, -m));  // the largest p, as computed below
-          corr = __bfloat162float(__float2bfloat16_rn(em)) - em;
-        }
         // p = 2^(s * scale - m) in pairs, written over this tile's S buffer as bf16 pairs, 64 keys
         // (32 columns) at a time, each half signalled to the MMA issuer as soon as it is in TMEM
         const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2), nm2 = pack2(-m, -m);
@@ -594,6 +589,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_st_wait();
           tc_fence_before();
           arrive_cluster(p_full_l + 8u * h);
+        }
+        float corr = 0.f;
+        if (mx > m) {
+          const float em = ex2_approx(fmaf(raw_max, p.scale_log2, -m));  // the largest p, as computed above
+          corr = __bfloat162float(__float2bfloat16_rn(em)) - em;
         }
         const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
         l = l * alpha + ((lo2(a2) + hi2(a2)) + corr);
