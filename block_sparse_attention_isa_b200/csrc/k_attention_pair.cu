@@ -45,9 +45,12 @@
 //    staggered instead of sharing the ex2 units at the same time;
 //  * the softmax writes P in two halves of 64 keys and signals each, so the P V
 //    MMAs of the first half run while the second half is exponentiated;
-//  * lazy rescaling (the running max moves only when it grows by more than 2^8),
-//    exact items first and Taylor items after in the static schedule; one pair
-//    of exponentials in eight on the FMA-pipe polynomial (exp2_poly.cuh);
+//  * work items from a per-call counter, exact items first and Taylor items
+//    after: the leader's producer takes each index and publishes it to both CTAs'
+//    roles through a ring in shared memory, so a pair that finishes its exact
+//    items early fills the end with the cheap Taylor items;
+//  * lazy rescaling (the running max moves only when it grows by more than 2^8);
+//    one pair of exponentials in eight on the FMA-pipe polynomial (exp2_poly.cuh);
 //  * every wait is bounded; on a timeout the CTA flags an error in the device
 //    error word and in the abort flags of both CTAs, lets its copies land,
 //    meets its peer at a cluster barrier and frees TMEM.
@@ -94,6 +97,8 @@ constexpr int kVHalf = kBN * 128;     // 16 KB: 128 keys x this CTA's 64 columns
 constexpr uint32_t kIdescQK = umma_idesc(1u, 256, kBN, 0, 0);
 constexpr uint32_t kIdescPV = umma_idesc(1u, 256, kD, 0, 1);
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kRing = 4;  // work items published ahead by the leader's producer
+constexpr int kItemFreeArrivals = 1 + 256 + 1 + 256;
 // Share of the exponentials computed by the FMA-pipe polynomial (exp2_poly.cuh) instead of
 // ex2: pair i of a row goes to the polynomial when (i % kPolyDen) < kPolyNum. One pair in eight
 // measured 1.5-2.5 % faster than none; two in eight slower again.
@@ -128,6 +133,7 @@ struct PairParams {
 struct PairExtra {
   float* lse;          // kLse: [BH, N] natural log of each row's softmax denominator
   const int32_t* sel;  // kRagged: [BH, k] kept context blocks
+  uint32_t* next;      // per-call work counter (zeroed with the control words)
 };
 
 struct Bars {
@@ -139,6 +145,12 @@ struct Bars {
   uint64_t p_full[2][2];  // leader: [slot][half], one arrival per softmax thread of both CTAs
   uint64_t o_done[2];     // [slot]: the P V MMAs of the slot's item are complete
   uint64_t drain;         // leader: every MMA is complete
+  // Work items, taken by the leader's producer from the per-call counter and published to both
+  // CTAs through a ring: item_full in each CTA (1 arrival), item_free in the leader (the
+  // leader's issuer and softmax threads, the peer's producer and softmax threads).
+  uint64_t item_full[kRing];
+  uint64_t item_free[kRing];
+  int item_ring[kRing];  // item index, or -1 past the last
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -149,20 +161,6 @@ constexpr int kOffV = kOffK + kStages * kKHalf;
 constexpr int kOffBar = kOffV + kStages * kVHalf;
 constexpr int kSmemAlloc = kOffBar + (int)sizeof(Bars) + 1024;
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
-
-// The k-th work item of CTA pair `pair`, or -1 past its last. Exact items all cost the same
-// and go round-robin over the pairs; when they do not divide evenly, the first E % npairs
-// pairs hold one more of them, so the (much cheaper) Taylor items go round-robin over the
-// other pairs only. Every role of both CTAs walks the same sequence.
-__device__ __forceinline__ int schedule(const PairParams& p, int pair, int npairs, int k) {
-  const int E = p.BH * p.items_e, T = p.BH * p.items_t;
-  const int n_exact = pair < E ? (E - pair + npairs - 1) / npairs : 0;
-  if (k < n_exact) return pair + k * npairs;
-  const int busy = E % npairs;
-  if (pair < busy) return -1;
-  const int g = (pair - busy) + (k - n_exact) * (npairs - busy);
-  return g < T ? E + g : -1;
-}
 
 // First token of query block i (source blocks from 0, context blocks from L_src) and its length.
 __device__ __forceinline__ int qblock_start(const PairParams& p, int i) {
@@ -189,6 +187,35 @@ __device__ __forceinline__ void add_col_bias(uint32_t (&r)[kCols], int base, int
 #pragma unroll
   for (int i = 0; i < kCols; ++i)
     if (i == c) r[i] = __float_as_uint(__uint_as_float(r[i]) + delta);
+}
+
+// Cluster-scope acquire wait (the peer CTA's item ring is written and signalled by the leader's
+// producer), bounded like mbar_wait_or_abort.
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_acq_cluster_or_abort(uint64_t* bar, uint32_t parity, const int* abort) {
+  const uint32_t a = smem_addr(bar);
+  if (mbar_try_wait_acq_cluster(a, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait_acq_cluster(a, parity)) return true;
+    if (*reinterpret_cast<const volatile int*>(abort) != 0) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+  }
+}
+__device__ __forceinline__ void arrive_cluster_release(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
 
 struct Item {
@@ -270,7 +297,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -283,6 +309,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&bars->item_full[i], 1);
+      mbar_init(&bars->item_free[i], kItemFreeArrivals);
     }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -321,7 +351,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t kv_full_l = map_to(&bars->kv_full[0], 0);
       uint32_t kv_it = 0, q_loads0 = 0, q_loads1 = 0;
       bool ok = true;
-      for (int k = 0, g = schedule(p, pair, npairs, 0); g >= 0 && ok; g = schedule(p, pair, npairs, ++k)) {
+      // Items in counter order: all exact items, then the (much cheaper) Taylor items, so a pair
+      // that finishes its exact work early fills the end with Taylor items.
+      for (uint32_t n = 0; ok; ++n) {
+        const uint32_t slot = n % kRing;
+        int g;
+        if (rank == 0) {
+          if (n >= kRing && !mbar_wait(&bars->item_free[slot], ((n / kRing) - 1) & 1)) {
+            raise_abort(bars, p.err, kErrProducer);
+            ok = false;
+            break;
+          }
+          g = (int)atomicAdd(x.next, 1u);
+          if (g >= p.total) g = -1;
+          *reinterpret_cast<volatile int*>(&bars->item_ring[slot]) = g;
+          store_cluster_u32(map_to(&bars->item_ring[slot], 1), (uint32_t)g);
+          mbar_arrive(&bars->item_full[slot]);
+          arrive_cluster_release(map_to(&bars->item_full[slot], 1));
+        } else {
+          if (!mbar_wait_acq_cluster_or_abort(&bars->item_full[slot], (n / kRing) & 1, &bars->abort_flag)) {
+            raise_abort(bars, p.err, kErrProducer);
+            ok = false;
+            break;
+          }
+          g = *reinterpret_cast<volatile int*>(&bars->item_ring[slot]);
+          arrive_cluster_release(map_to(&bars->item_free[slot], 0));
+        }
+        if (g < 0) break;
         const Item it = decode_item(p, g);
         for (int t = 0; t < it.nslots; ++t) {
           // slot t's Q buffer is free once the S MMAs of the last item that used it are complete
@@ -444,7 +500,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         return true;
       };
-      for (int k = 0, g = schedule(p, pair, npairs, 0); g >= 0 && ok; g = schedule(p, pair, npairs, ++k)) {
+      for (uint32_t n = 0; ok; ++n) {
+        const uint32_t slot = n % kRing;
+        if (!wait(&bars->item_full[slot], (n / kRing) & 1)) break;
+        const int g = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&bars->item_ring[slot]), 0);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->item_free[slot]);
+        if (g < 0) break;
         const Item it = decode_item(p, g);
         const int ns = it.nslots;
 #pragma unroll
@@ -508,7 +570,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t seq = 0, items = 0;
     bool ok = true;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-    for (int k = 0, g = schedule(p, pair, npairs, 0); g >= 0 && ok; g = schedule(p, pair, npairs, ++k)) {
+    const uint32_t item_free_l = map_to(&bars->item_free[0], 0);
+    for (uint32_t n = 0; ok; ++n) {
+      const uint32_t slot = n % kRing;
+      {
+        bool got = rank == 0 ? mbar_wait_or_abort(&bars->item_full[slot], (n / kRing) & 1, &bars->abort_flag)
+                             : mbar_wait_acq_cluster_or_abort(&bars->item_full[slot], (n / kRing) & 1,
+                                                              &bars->abort_flag);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) {
+          if (lane == 0) raise_abort(bars, p.err, kErrSoftmax);
+          ok = false;
+          break;
+        }
+      }
+      const int g = *reinterpret_cast<volatile int*>(&bars->item_ring[slot]);
+      if (rank == 0) mbar_arrive(&bars->item_free[slot]);
+      else arrive_cluster_release(item_free_l + 8u * slot);
+      if (g < 0) break;
       const Item it = decode_item(p, g);
       if (t >= it.nslots) continue;
       const bool cs = kRagged ? short_ctx_kept(p, x.sel, it.bh) : false;
@@ -739,7 +818,8 @@ cudaError_t launch_attention_pair(const void* q, const void* k, const void* v, v
     if (dev >= 0 && dev < 64) cached_pairs[dev] = pairs;
   }
   if (pairs > p.total) pairs = p.total;
-  kern<<<2 * pairs, kThreads, kSmemAlloc, s>>>(tq, tk, tks, tv, tvs, tkc, tvc, p, PairExtra{w.lse, w.sel});
+  kern<<<2 * pairs, kThreads, kSmemAlloc, s>>>(tq, tk, tks, tv, tvs, tkc, tvc, p,
+                                                PairExtra{w.lse, w.sel, w.ctrl + kCtrlPairNext});
   if (n_ctas) *n_ctas = 2 * pairs;
   return cudaGetLastError();
 }
