@@ -85,6 +85,7 @@ enum : int {
   kCtrlGridBarrier = 1,
   kCtrlMixedNext = 2,  // next work item of the mixed Taylor kernel (dynamic schedule)
   kCtrlPairNext = 3,   // next work item of the CTA-pair attention kernel (dynamic schedule)
+  kCtrlBwdNext = 4,    // [3]: next work item of the three backward launches (dynamic schedule)
 };
 
 // Floats of the pooling kernel's per-item partial sums for these sizes.

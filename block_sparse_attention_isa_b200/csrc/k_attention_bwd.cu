@@ -92,12 +92,19 @@ struct BwdParams {
   float log2_b;           // the Taylor rows' weight b, dropped from their exponents
 };
 
+constexpr int kRing = 4;
+
 struct Bars {
   uint64_t a_full, a_empty;
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], p_full[2];
   uint64_t acc_full, acc_empty;
   uint64_t drain;
+  // Work items from the per-launch counter (exact items first, then Taylor items), published by
+  // the producer lane: item_full (1 arrival), item_free (the issuer and the 256 elementwise threads).
+  uint64_t item_full[kRing];
+  uint64_t item_free[kRing];
+  int item_ring[kRing];  // item index, or -1 past the last
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -197,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_ksel, const __grid_constant__ CUtensorMap tm_vsel,
                          const __grid_constant__ CUtensorMap tm_kcn, const __grid_constant__ CUtensorMap tm_vcn,
-                         const BwdParams p) {
+                         const BwdParams p, uint32_t* next) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA1 = smem + kOffA1;
@@ -220,6 +227,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->acc_full, 1);
     mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->drain, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&bars->item_full[i], 1);
+      mbar_init(&bars->item_free[i], 257);
+    }
     bars->abort_flag = 0;
     mbar_fence_init();
   }
@@ -270,7 +281,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 2; ++c) tma_load_3d(dst + c * ch, grad ? &tm_do : &tm_q, bar, c * 64, tok, bh);
       };
-      for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x) {
+      for (uint32_t n = 0; ok; ++n) {
+        const uint32_t slot = n % kRing;
+        if (n >= kRing && !mbar_wait(&bars->item_free[slot], ((n / kRing) - 1) & 1)) {
+          raise_abort(bars, p.err, kErrProducer);
+          ok = false;
+          break;
+        }
+        int g = (int)atomicAdd(next, 1u);
+        if (g >= p.total) g = -1;
+        *reinterpret_cast<volatile int*>(&bars->item_ring[slot]) = g;
+        mbar_arrive(&bars->item_full[slot]);
+        if (g < 0) break;
         const Item it = decode_item<kDKDV>(p, g);
         if (it.c_end <= it.c_begin) continue;  // nothing to accumulate (every role skips it)
         if (n_items > 0 && !mbar_wait(&bars->a_empty, (n_items - 1) & 1)) {
@@ -361,7 +383,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             (acc | (uint32_t)s) != 0 ? 1u : 0u);
       };
       const uint32_t t_s = tmem, t_t = tmem + 128, t_acc0 = tmem + 256, t_acc1 = tmem + 384;
-      for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x) {
+      for (uint32_t n = 0; ok; ++n) {
+        const uint32_t slot = n % kRing;
+        if (!wait(&bars->item_full[slot], (n / kRing) & 1)) break;
+        const int g = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&bars->item_ring[slot]), 0);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->item_free[slot]);
+        if (g < 0) break;
         const Item it = decode_item<kDKDV>(p, g);
         if (it.c_end <= it.c_begin) continue;
         if (!wait(&bars->a_full, n_items & 1)) break;
@@ -428,7 +456,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t n_items = 0, tile_it = 0, ct = 0;
     bool ok = true;
     const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2);
-    for (int g = blockIdx.x; g < p.total && ok; g += gridDim.x) {
+    for (uint32_t n = 0; ok; ++n) {
+      const uint32_t slot = n % kRing;
+      if (!warp_wait(bars, &bars->item_full[slot], (n / kRing) & 1, p.err)) { ok = false; break; }
+      const int g = *reinterpret_cast<volatile int*>(&bars->item_ring[slot]);
+      mbar_arrive(&bars->item_free[slot]);
+      if (g < 0) break;
       const Item it = decode_item<kDKDV>(p, g);
       const int nc = it.c_end - it.c_begin;
       const float path_off = it.kind == 1 ? p.log2_b : 0.f;  // the Taylor exponents omit the weight b
@@ -623,7 +656,7 @@ __global__ void bwd_delta_kernel(const __nv_bfloat16* __restrict__ dout, const _
 
 template <bool kDKDV>
 cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* dout, const Plan& pl, const Work& w,
-                       BwdParams p, cudaStream_t s) {
+                       BwdParams p, uint32_t* next, cudaStream_t s) {
   p.total = p.kind_split + pl.BH * p.items_t;
   if (p.total == 0) return cudaSuccess;
   CUtensorMap tq, tdo, tk, tv, tks, tvs, tkc, tvc;
@@ -645,7 +678,7 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* 
   if (e != cudaSuccess) return e;
   int grid = device_sm_count();
   if (grid > p.total) grid = p.total;
-  kern<<<grid, kThreads, kSmemAlloc, s>>>(tq, tdo, tk, tv, tks, tvs, tkc, tvc, p);
+  kern<<<grid, kThreads, kSmemAlloc, s>>>(tq, tdo, tk, tv, tks, tvs, tkc, tvc, p, next);
   return cudaGetLastError();
 }
 
@@ -694,6 +727,7 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
   p.dk = dk;
   p.dv = dv;
   p.err = w.ctrl;
+  if ((e = cudaMemsetAsync(w.ctrl + kCtrlBwdNext, 0, 3 * sizeof(uint32_t), s)) != cudaSuccess) return e;
   p.BH = pl.BH;
   p.N = pl.N;
   p.b = pl.b;
@@ -714,7 +748,7 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
     d.items_t = (pl.n_flat * pl.b + kBM - 1) / kBM;
     d.kind_split = pl.BH * d.items_e;
     d.chunks = 1;
-    if ((e = launch_bwd<false>(q, k, v, dout, pl, w, d, s)) != cudaSuccess) return e;
+    if ((e = launch_bwd<false>(q, k, v, dout, pl, w, d, w.ctrl + kCtrlBwdNext, s)) != cudaSuccess) return e;
   }
   // dK/dV of the Taylor path over the pooled rows: column ranges split so that the grid fills
   // the GPU, partial sums added into dKc / dVc
@@ -731,7 +765,7 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
     d.chunks = chunks;
     d.items_t = row_tiles * chunks;
     d.kind_split = 0;
-    if ((e = launch_bwd<true>(q, k, v, dout, pl, w, d, s)) != cudaSuccess) return e;
+    if ((e = launch_bwd<true>(q, k, v, dout, pl, w, d, w.ctrl + kCtrlBwdNext + 1, s)) != cudaSuccess) return e;
   }
   // dK/dV of the exact path over the rows of K_new, plus the Taylor spread, written to dK / dV
   {
@@ -742,7 +776,7 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
     d.items_t = 0;
     d.kind_split = pl.BH * d.items_e;
     d.chunks = 1;
-    if ((e = launch_bwd<true>(q, k, v, dout, pl, w, d, s)) != cudaSuccess) return e;
+    if ((e = launch_bwd<true>(q, k, v, dout, pl, w, d, w.ctrl + kCtrlBwdNext + 2, s)) != cudaSuccess) return e;
   }
   return cudaSuccess;
 }
