@@ -339,7 +339,11 @@ ISA_API size_t isa_backward_workspace_bytes(int B, int H, int L_src, int L_ctx, 
  *   q, k, v, out, lse  the forward call's inputs and outputs (isa_forward_train)
  *   dout               [B, H, N, D] gradient of the output
  *   dq, dk, dv         [B, H, N, D] outputs (bfloat16), not overlapping the inputs
- *   fwd_workspace      the workspace of that isa_forward_train call, untouched since
+ *   fwd_workspace      the workspace of that isa_forward_train call, untouched since;
+ *                      the call reads its decisions and pooled rows and uses three of
+ *                      its control words as work counters, so two backward calls on one
+ *                      forward workspace must not run at the same time (in stream order
+ *                      they may run any number of times)
  *   bwd_workspace      at least isa_backward_workspace_bytes(), 256-byte aligned
  * Other arguments must equal the forward call's. Asynchronous, no allocation. A
  * kernel wait that gives up is reported by isa_device_status(fwd_workspace).
